@@ -1,0 +1,175 @@
+"""Seeded synthetic inputs shaped like the attention of Wan 2.1 14B and Mochi 1.
+
+This module holds input construction only (random numbers, positional
+features, random block masks); none of CalibAtt's arithmetic lives here. Both
+the CUDA path's tests/benchmark and the oracle read the same tensors from it.
+
+Recipe (the pages measure on real models and prompts; these stand in for the
+attention inputs of those models at the same shapes):
+
+* tokens of a latent video F x H x W, row-major within a frame, frames
+  consecutive: t = f*H*W + r*W + c;
+* q_i = g_i + 2 e(pos_i), k_j = h_j + 2 e(pos_j), with g, h, v ~ N(0, 1) drawn
+  per (config, input, head) and e = 64 random Fourier features
+  cos(2 pi w_m . pos + b_m) of the normalised position pos = (f/F, r/H, c/W),
+  zero-padded to d = 128. w_m ~ N(0, sigma_h^2 I_3) and b_m ~ U[0, 2 pi) are
+  drawn per head only, fixed across inputs, which is what makes the block
+  structure stable from one input to the next;
+* values are rounded to bf16 (round to nearest even).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+D_HEAD = 128
+BLOCK = 128
+N_FEAT = 64
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    F: int
+    H: int
+    W: int
+    heads: int
+    repeat_heads: tuple = ()
+    k_anchor: int = 5
+    config_id: int = 0
+    sigma_range: tuple = (1.0, 3.0)
+
+    @property
+    def n(self) -> int:
+        return self.F * self.H * self.W
+
+    @property
+    def nb(self) -> int:
+        return (self.n + BLOCK - 1) // BLOCK
+
+
+# The five workloads. Repeat heads: one head in five on Wan-720p (8 of 40) and
+# one in six on Mochi (4 of 24).
+WORKLOADS = {
+    "tiny": Workload("tiny", 16, 8, 16, 1, (), 5, 1, (1.5, 1.5)),
+    "wan480": Workload("wan480", 21, 30, 52, 40, (), 5, 2),
+    "wan720": Workload("wan720", 21, 45, 80, 40, tuple(h for h in range(40) if h % 5 == 4), 5, 3),
+    "mochi480": Workload("mochi480", 28, 30, 53, 24, tuple(h for h in range(24) if h % 6 == 5), 5, 4),
+    "calib720": Workload("calib720", 21, 45, 80, 40, (), 5, 5),
+}
+
+
+def _seed(*parts: int) -> int:
+    ss = np.random.SeedSequence([int(p) & 0xFFFFFFFF for p in parts])
+    return int(ss.generate_state(1, dtype=np.uint64)[0] & 0x7FFFFFFFFFFFFFFF)
+
+
+def positions(F: int, H: int, W: int) -> np.ndarray:
+    """Normalised (f/F, r/H, c/W) of every token, [F*H*W, 3] float64."""
+    f, r, c = np.meshgrid(np.arange(F) / F, np.arange(H) / H, np.arange(W) / W, indexing="ij")
+    return np.stack([f.ravel(), r.ravel(), c.ravel()], axis=1)
+
+
+def head_sigma(wl: Workload, head: int) -> float:
+    lo, hi = wl.sigma_range
+    if lo == hi:
+        return float(lo)
+    u = np.random.default_rng(_seed(wl.config_id, 77, head)).random()
+    return float(math.exp(math.log(lo) + u * (math.log(hi) - math.log(lo))))
+
+
+def fourier_features(wl: Workload, head: int) -> torch.Tensor:
+    """e(pos) for every token of one head, zero-padded to d: [n, 128] float32."""
+    rng = np.random.default_rng(_seed(wl.config_id, 11, head))
+    sigma = head_sigma(wl, head)
+    w = rng.normal(0.0, sigma, size=(N_FEAT, 3))
+    b = rng.uniform(0.0, 2.0 * math.pi, size=(N_FEAT,))
+    pos = positions(wl.F, wl.H, wl.W)
+    e = np.cos(2.0 * math.pi * pos @ w.T + b)
+    out = torch.zeros((wl.n, D_HEAD), dtype=torch.float32)
+    out[:, :N_FEAT] = torch.from_numpy(e.astype(np.float32))
+    return out
+
+
+def _normal(shape, seed: int) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return torch.randn(shape, generator=g, dtype=torch.float32)
+
+
+def qkv(wl: Workload, input_idx: int, heads=None, with_v: bool = True):
+    """bf16 CPU tensors q, k (and v), [len(heads)][n][128] for one input."""
+    heads = list(range(wl.heads)) if heads is None else list(heads)
+    qs, ks, vs = [], [], []
+    for h in heads:
+        e = fourier_features(wl, h)
+        qs.append((_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 1)) + 2.0 * e).to(torch.bfloat16))
+        ks.append((_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 2)) + 2.0 * e).to(torch.bfloat16))
+        if with_v:
+            vs.append(_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 3)).to(torch.bfloat16))
+    q = torch.stack(qs)
+    k = torch.stack(ks)
+    v = torch.stack(vs) if with_v else None
+    return q, k, v
+
+
+def plain_qkv(heads: int, n: int, seed: int, d: int = D_HEAD, std: float = 1.0):
+    """Unstructured bf16 N(0, std^2) q, k, v [heads][n][d] (edge-case tests)."""
+    out = []
+    for i in range(3):
+        out.append((_normal((heads, n, d), _seed(seed, 900 + i)) * std).to(torch.bfloat16))
+    return tuple(out)
+
+
+def random_block_masks(wl: Workload, target_keep: float = 0.375, seed: int = 3000) -> np.ndarray:
+    """Random per-head block masks [heads][nb][nb] uint8 (Wan-720p workload).
+
+    Keep probability per head p_h ~ Beta(2, 3); each block is kept with
+    probability min(1, c p_h); the diagonal block and the key blocks of the
+    first frame are always kept; c is solved so that the expected kept
+    fraction over the non-repeat heads equals ``target_keep``.
+    """
+    nb = wl.nb
+    first_frame_blocks = (wl.H * wl.W + BLOCK - 1) // BLOCK
+    forced = np.zeros((nb, nb), bool)
+    forced[:, :first_frame_blocks] = True
+    forced[np.arange(nb), np.arange(nb)] = True
+    n_forced = int(forced.sum())
+    p = np.array([np.random.default_rng(seed + h).beta(2.0, 3.0) for h in range(wl.heads)])
+    active = [h for h in range(wl.heads) if h not in wl.repeat_heads]
+
+    def expected(c):
+        return np.mean([(n_forced + (nb * nb - n_forced) * min(1.0, c * p[h])) / (nb * nb) for h in active])
+
+    lo, hi = 0.0, 1.0
+    while expected(hi) < target_keep and hi < 1e6:
+        hi *= 2
+    for _ in range(100):
+        mid = 0.5 * (lo + hi)
+        if expected(mid) < target_keep:
+            lo = mid
+        else:
+            hi = mid
+    c = 0.5 * (lo + hi)
+    masks = np.zeros((wl.heads, nb, nb), np.uint8)
+    for h in range(wl.heads):
+        rng = np.random.default_rng(seed + 100 + h)
+        keep = rng.random((nb, nb)) < min(1.0, c * p[h])
+        masks[h] = (keep | forced).astype(np.uint8)
+    return masks
+
+
+def random_mask(heads: int, nb: int, keep: float, seed: int) -> np.ndarray:
+    """Plain Bernoulli(keep) block mask with the diagonal kept (tests)."""
+    rng = np.random.default_rng(_seed(seed, 5))
+    m = (rng.random((heads, nb, nb)) < keep).astype(np.uint8)
+    m[:, np.arange(nb), np.arange(nb)] = 1
+    return m
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> uint16 numpy array of its bit patterns."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
