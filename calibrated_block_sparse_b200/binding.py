@@ -1,0 +1,285 @@
+"""ctypes binding of libcalibatt (include/calibatt.h): argument marshalling only.
+
+Every step of the hot path runs in the CUDA library; this module turns torch
+tensors into pointers, sizes and the current CUDA stream, allocates outputs
+with torch when the caller does not pass them, and raises ``CalibattError``
+on a nonzero status. There is no CPU fallback: if the library is missing the
+import of a compute function fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+_lock = threading.Lock()
+_lib = None
+
+BLOCK = 128
+HEAD_DIM = 128
+
+
+class CalibattError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} ({code})" if what else f"{strerror(code)} ({code})")
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load(build_if_missing: bool = False):
+    """Load libcalibatt.so (optionally building it first). Raises if absent."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if build_if_missing and _build.needs_build():
+            _build.build()
+        if not os.path.exists(path):
+            raise ImportError(f"libcalibatt.so is not built ({path}); run python -m calibrated_block_sparse_b200.build")
+        lib = ctypes.CDLL(path)
+        P, i32, i64, f32, f64, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                                     ctypes.c_double, ctypes.c_size_t)
+        sig = {
+            "calibatt_strerror": (ctypes.c_char_p, [i32]),
+            "calibatt_version": (i32, []),
+            "calibatt_get_status": (i32, [P]),
+            "calibatt_eps_schedule": (f64, [f64, f64, f64, f64, f64]),
+            "calibatt_validate_csr": (i32, [P, P, i32, i32, i64]),
+            "calibatt_build_plan": (i32, [P, i32, i32, P, P, P]),
+            "calibatt_anchor_rows": (i32, [i32, i32, P]),
+            "calibatt_rho_threshold": (i32, [i32, f64, P]),
+            "calibatt_sparse_attn_fwd": (i32, [P, P, P, i32, i32, i32, f32, P, P, i64, P, i32, P, P, P]),
+            "calibatt_repeat_workspace_size": (sz, [i32, i32, i32, i32, i32]),
+            "calibatt_repeat_attn_fwd": (i32, [P, P, P, i32, i32, i32, i32, i32, i32, f32, P, i32, P, P, P, sz, P]),
+            "calibatt_block_energy": (i32, [P, P, i32, i32, i32, f32, P, P, i32, f64, P, P, P, P]),
+            "calibatt_select_mask": (i32, [P, i32, i32, f64, P, P, P, P]),
+            "calibatt_accumulate_masks": (i32, [P, i64, P, P]),
+            "calibatt_aggregate_workspace_size": (sz, [i32, i32]),
+            "calibatt_aggregate_masks": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P, sz, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def strerror(code: int) -> str:
+    return load().calibatt_strerror(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise CalibattError(rc, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return ctypes.c_void_p(t.ctypes.data)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda_tensor(t, dtype, name):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise TypeError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    return t
+
+
+def _bhnd(q, name="q"):
+    _cuda_tensor(q, torch.bfloat16, name)
+    if q.dim() != 3 or q.shape[-1] != HEAD_DIM:
+        raise ValueError(f"{name} must be [heads][n][{HEAD_DIM}]")
+    return q.shape[0], q.shape[1]
+
+
+# ------------------------------------------------------------------ host helpers
+
+def get_status(stream=None) -> int:
+    return load().calibatt_get_status(_stream(stream))
+
+
+def check_status(stream=None, what="kernel"):
+    _check(get_status(stream), what)
+
+
+def eps_schedule(A, C, k, t, T) -> float:
+    return load().calibatt_eps_schedule(float(A), float(C), float(k), float(t), float(T))
+
+
+def validate_csr(row_ptr: np.ndarray, col_idx: np.ndarray, heads: int, nb: int) -> int:
+    rp = np.ascontiguousarray(row_ptr, np.int32)
+    ci = np.ascontiguousarray(col_idx, np.int32)
+    return load().calibatt_validate_csr(_ptr(rp), _ptr(ci) if ci.size else None, heads, nb, int(ci.size))
+
+
+def build_plan(row_ptr: np.ndarray, heads: int, nb: int, head_active=None) -> np.ndarray:
+    rp = np.ascontiguousarray(row_ptr, np.int32)
+    ha = None if head_active is None else np.ascontiguousarray(head_active, np.uint8)
+    out = np.empty(heads * nb, np.int32)
+    n = np.zeros(1, np.int32)
+    _check(load().calibatt_build_plan(_ptr(rp), heads, nb, _ptr(ha), _ptr(out), _ptr(n)), "build_plan")
+    return out[: int(n[0])].copy()
+
+
+def anchor_rows(H: int, k_anchor: int) -> np.ndarray:
+    out = np.empty(k_anchor, np.int32)
+    _check(load().calibatt_anchor_rows(H, k_anchor, _ptr(out)), "anchor_rows")
+    return out
+
+
+def rho_threshold(n_inputs: int, rho: float) -> int:
+    out = np.zeros(1, np.int32)
+    _check(load().calibatt_rho_threshold(int(n_inputs), float(rho), _ptr(out)), "rho_threshold")
+    return int(out[0])
+
+
+# ------------------------------------------------------------------ inference
+
+def sparse_attn_fwd(q, k, v, row_ptr, col_idx, work_list, o=None, lse=None, scale=None, want_lse=True,
+                    stream=None):
+    """Block-sparse attention over a skip list; returns (o, lse)."""
+    heads, n = _bhnd(q)
+    _bhnd(k, "k")
+    _bhnd(v, "v")
+    _cuda_tensor(row_ptr, torch.int32, "row_ptr")
+    _cuda_tensor(col_idx, torch.int32, "col_idx")
+    _cuda_tensor(work_list, torch.int32, "work_list")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((heads, n), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = load().calibatt_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), heads, n, HEAD_DIM, scale, _ptr(row_ptr),
+                                         _ptr(col_idx) if col_idx.numel() else None, col_idx.numel(),
+                                         _ptr(work_list) if work_list.numel() else None, work_list.numel(),
+                                         _ptr(o), _ptr(lse), _stream(stream))
+    _check(rc, "calibatt_sparse_attn_fwd")
+    return o, lse
+
+
+def repeat_workspace_size(n_rep, F, H, W, k_anchor=5) -> int:
+    return load().calibatt_repeat_workspace_size(n_rep, F, H, W, k_anchor)
+
+
+def repeat_attn_fwd(q, k, v, F, H, W, rep_heads, k_anchor=5, o=None, lse=None, ws=None, scale=None,
+                    want_lse=True, stream=None):
+    """Anchor-row attention of repeated heads broadcast to every row; returns (o, lse)."""
+    heads, n = _bhnd(q)
+    _cuda_tensor(rep_heads, torch.int32, "rep_heads")
+    n_rep = rep_heads.numel()
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((heads, n), dtype=torch.float32, device=q.device)
+    need = repeat_workspace_size(max(n_rep, 1), F, H, W, k_anchor)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = load().calibatt_repeat_attn_fwd(_ptr(q), _ptr(k), _ptr(v), heads, F, H, W, HEAD_DIM, k_anchor, scale,
+                                         _ptr(rep_heads), n_rep, _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                                         _stream(stream))
+    _check(rc, "calibatt_repeat_attn_fwd")
+    return o, lse
+
+
+# ------------------------------------------------------------------ calibration
+
+def block_energy(q, k, eps=None, energy=True, mask=None, kept=None, counts=None, lse_ws=None, scale=None,
+                 stream=None):
+    """Block energy of one input; with eps, fused greedy selection too.
+
+    Returns (energy or None, mask, kept, counts) — the outputs that were requested.
+    """
+    heads, n = _bhnd(q)
+    nb = (n + BLOCK - 1) // BLOCK
+    dev = q.device
+    if lse_ws is None:
+        lse_ws = torch.empty((heads, nb * BLOCK), dtype=torch.float32, device=dev)
+    e = None
+    if energy is True:
+        e = torch.empty((heads, nb, nb), dtype=torch.float32, device=dev)
+    elif isinstance(energy, torch.Tensor):
+        e = energy
+    fuse = eps is not None
+    if fuse and mask is None and kept is None and counts is None:
+        mask = torch.empty((heads, nb, nb), dtype=torch.uint8, device=dev)
+        kept = torch.empty((heads, nb), dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = load().calibatt_block_energy(_ptr(q), _ptr(k), heads, n, HEAD_DIM, scale, _ptr(lse_ws), _ptr(e),
+                                      1 if fuse else 0, float(eps) if fuse else 0.0, _ptr(mask), _ptr(kept),
+                                      _ptr(counts), _stream(stream))
+    _check(rc, "calibatt_block_energy")
+    return e, mask, kept, counts
+
+
+def select_mask(energy, eps, mask=True, kept=True, counts=None, stream=None):
+    """Greedy eps selection on [heads][nb][nb] energies; returns (mask, kept, counts)."""
+    _cuda_tensor(energy, torch.float32, "energy")
+    heads, nb, _ = energy.shape
+    dev = energy.device
+    if mask is True:
+        mask = torch.empty((heads, nb, nb), dtype=torch.uint8, device=dev)
+    elif mask is False:
+        mask = None
+    if kept is True:
+        kept = torch.empty((heads, nb), dtype=torch.int32, device=dev)
+    elif kept is False:
+        kept = None
+    rc = load().calibatt_select_mask(_ptr(energy), heads, nb, float(eps), _ptr(mask), _ptr(kept), _ptr(counts),
+                                     _stream(stream))
+    _check(rc, "calibatt_select_mask")
+    return mask, kept, counts
+
+
+def accumulate_masks(mask, counts, stream=None):
+    _cuda_tensor(mask, torch.uint8, "mask")
+    _cuda_tensor(counts, torch.uint16, "counts")
+    rc = load().calibatt_accumulate_masks(_ptr(mask), mask.numel(), _ptr(counts), _stream(stream))
+    _check(rc, "calibatt_accumulate_masks")
+    return counts
+
+
+def aggregate_masks(counts, n_inputs, rho=0.5, nnz_cap=None, ws=None, stream=None, trim=True):
+    """Binarise counts at rho and build the CSR skip list.
+
+    Returns (mask, row_ptr, col_idx, nnz). With trim, col_idx is cut to nnz
+    (one device-to-host read of the total)."""
+    _cuda_tensor(counts, torch.uint16, "counts")
+    heads, nb, _ = counts.shape
+    dev = counts.device
+    if nnz_cap is None:
+        nnz_cap = heads * nb * nb
+    mask = torch.empty((heads, nb, nb), dtype=torch.uint8, device=dev)
+    row_ptr = torch.empty(heads * nb + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(int(nnz_cap), 1), dtype=torch.int32, device=dev)
+    nnz = torch.zeros(1, dtype=torch.int64, device=dev)
+    need = load().calibatt_aggregate_workspace_size(heads, nb)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    rc = load().calibatt_aggregate_masks(_ptr(counts), int(n_inputs), heads, nb, float(rho), _ptr(mask),
+                                         _ptr(row_ptr), _ptr(col_idx), int(nnz_cap), _ptr(nnz), _ptr(ws),
+                                         ws.numel(), _stream(stream))
+    _check(rc, "calibatt_aggregate_masks")
+    if trim:
+        total = int(nnz.item())
+        col_idx = col_idx[:total]
+    return mask, row_ptr, col_idx, nnz

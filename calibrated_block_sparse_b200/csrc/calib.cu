@@ -1,0 +1,185 @@
+// Bandwidth-bound calibration and packing kernels: standalone greedy eps
+// selection, mask accumulation over inputs, rho aggregation into a CSR skip
+// list, and the anchor-row query gather of repeated heads.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "calibatt.h"
+#include "kernels.h"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace calibatt {
+
+
+// ------------------------------------------------------------------ selection
+// One 128-thread CTA per block-row of energies.
+__global__ void __launch_bounds__(128) select_kernel(const float* __restrict__ energy, int nb, long long eps_fx,
+                                                     uint8_t* mask, int32_t* kept, uint16_t* counts) {
+  __shared__ float e_row[1024];
+  __shared__ __align__(16) uint8_t aux[4096];
+  __shared__ unsigned long long keys[1024];
+  const int64_t row = blockIdx.x;
+  const float* src = energy + row * nb;
+  for (int c = threadIdx.x; c < nb; c += 128) e_row[c] = src[c];
+  __syncthreads();
+  SelectOut out{mask ? mask + row * nb : nullptr, kept ? kept + row : nullptr, counts ? counts + row * nb : nullptr};
+  select_row(e_row, nb, eps_fx, aux, keys, threadIdx.x, 128, 1, out);
+}
+
+// ------------------------------------------------------------------ accumulation
+__global__ void accumulate_kernel(const uint8_t* __restrict__ mask, int64_t cells, uint16_t* counts) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < cells; i += stride) {
+    const uint16_t c = counts[i];
+    if (mask[i] && c != 0xFFFFu) counts[i] = c + 1;
+  }
+}
+
+// ------------------------------------------------------------------ aggregation
+// Pass 1: one warp per (head, block-row): binarise counts >= threshold, write
+// the mask row and the row's kept count.
+__global__ void binarize_kernel(const uint16_t* __restrict__ counts, int64_t rows, int nb, int threshold,
+                                uint8_t* mask, int32_t* row_cnt) {
+  const int64_t row = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint16_t* src = counts + row * nb;
+  uint8_t* dst = mask + row * nb;
+  int cnt = 0;
+  for (int c = lane; c < nb; c += 32) {
+    const uint8_t k = src[c] >= threshold ? 1 : 0;
+    dst[c] = k;
+    cnt += k;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) row_cnt[row] = cnt;
+}
+
+// Pass 2: a single CTA turns the row counts into the exclusive prefix row_ptr
+// (global offsets) and the total.
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ row_cnt, int64_t rows,
+                                                    int32_t* row_ptr, int64_t nnz_cap, int64_t* nnz_out,
+                                                    int* status) {
+  __shared__ long long warp_tot[32];
+  __shared__ long long carry_s;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  long long carry = 0;
+  for (int64_t base = 0; base < rows; base += 1024) {
+    const int64_t i = base + tid;
+    const long long v = i < rows ? row_cnt[i] : 0;
+    long long incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    __syncthreads();
+    long long before = carry;
+    for (int ww = 0; ww < w; ++ww) before += warp_tot[ww];
+    if (i < rows) row_ptr[i] = static_cast<int32_t>(before + incl - v);
+    if (tid == 1023) carry_s = before + incl;
+    __syncthreads();
+    carry = carry_s;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    row_ptr[rows] = static_cast<int32_t>(carry);
+    *nnz_out = carry;
+    if (carry > nnz_cap) record_error(status, CALIBATT_ERR_CAPACITY);
+  }
+}
+
+// Pass 3: one warp per row writes the kept columns in ascending order.
+__global__ void compact_kernel(const uint8_t* __restrict__ mask, int64_t rows, int nb,
+                               const int32_t* __restrict__ row_ptr, int32_t* col_idx, int64_t nnz_cap) {
+  const int64_t row = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint8_t* src = mask + row * nb;
+  int64_t pos = row_ptr[row];
+  for (int c0 = 0; c0 < nb; c0 += 32) {
+    const int c = c0 + lane;
+    const bool k = c < nb && src[c];
+    const uint32_t bal = __ballot_sync(0xffffffffu, k);
+    if (k) {
+      const int64_t at = pos + __popc(bal & ((1u << lane) - 1u));
+      if (at < nnz_cap) col_idx[at] = c;
+    }
+    pos += __popc(bal);
+  }
+}
+
+// ------------------------------------------------------------------ anchor gather
+// Packs the anchor-row queries of repeated heads: packed row q = f*(k*W) +
+// j*W + c of head i is token f*H*W + anchors[j]*W + c of head rep_heads[i].
+// 16 threads move one 256-byte row.
+__global__ void gather_anchor_kernel(const uint4* __restrict__ q, int n, const int32_t* __restrict__ rep_heads,
+                                     int n_rep, int H, int W, int k_anchor, AnchorTable tab, uint4* out,
+                                     int heads, int* status) {
+  const int64_t per_head = static_cast<int64_t>(n / (H * W)) * k_anchor * W;
+  const int64_t total = per_head * n_rep * 16;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total; t += stride) {
+    const int part = static_cast<int>(t & 15);
+    const int64_t prow = t >> 4;
+    const int i = static_cast<int>(prow / per_head);
+    const int64_t qi = prow % per_head;
+    const int kw = k_anchor * W;
+    const int64_t f = qi / kw;
+    const int rem = static_cast<int>(qi % kw);
+    const int j = rem / W, c = rem % W;
+    int h = rep_heads[i];
+    if (h < 0 || h >= heads) {
+      record_error(status, CALIBATT_ERR_ARG);
+      h = 0;
+    }
+    const int64_t tok = f * H * W + static_cast<int64_t>(tab.anchor[j]) * W + c;
+    out[prow * 16 + part] = q[(static_cast<int64_t>(h) * n + tok) * 16 + part];
+  }
+}
+
+}  // namespace calibatt
+
+namespace calibatt {
+
+int launch_select(const float* energy, int64_t rows, int nb, long long eps_fx, uint8_t* mask, int32_t* kept,
+                  uint16_t* counts, cudaStream_t stream) {
+  if (rows <= 0) return CALIBATT_OK;
+  select_kernel<<<static_cast<unsigned>(rows), 128, 0, stream>>>(energy, nb, eps_fx, mask, kept, counts);
+  return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
+}
+
+int launch_accumulate(const uint8_t* mask, int64_t cells, uint16_t* counts, cudaStream_t stream) {
+  if (cells <= 0) return CALIBATT_OK;
+  int64_t blocks = (cells + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  accumulate_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(mask, cells, counts);
+  return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
+}
+
+int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold, uint8_t* mask, int32_t* row_ptr,
+                     int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* row_cnt, int* status,
+                     cudaStream_t stream) {
+  const unsigned warps_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  binarize_kernel<<<warps_blocks, 256, 0, stream>>>(counts, rows, nb, threshold, mask, row_cnt);
+  scan_kernel<<<1, 1024, 0, stream>>>(row_cnt, rows, row_ptr, nnz_cap, nnz, status);
+  compact_kernel<<<warps_blocks, 256, 0, stream>>>(mask, rows, nb, row_ptr, col_idx, nnz_cap);
+  return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
+}
+
+int launch_gather(const void* q, int n, int heads, const int32_t* rep_heads, int n_rep, int H, int W, int k_anchor,
+                  const AnchorTable& tab, void* out, int* status, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(n / (H * W)) * k_anchor * W * n_rep * 16;
+  if (total <= 0) return CALIBATT_OK;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  gather_anchor_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const uint4*>(q), n, rep_heads, n_rep, H, W, k_anchor, tab, static_cast<uint4*>(out), heads, status);
+  return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
+}
+
+}  // namespace calibatt

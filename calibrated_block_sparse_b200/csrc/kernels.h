@@ -1,0 +1,65 @@
+// Internal interface between the C-ABI entry points and the CUDA kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace calibatt {
+
+constexpr int kMaxAnchors = 64;
+
+// Parameters of the persistent tensor-core attention kernel (all modes).
+struct KernelParams {
+  int n_q;        // query rows per head in the Q tensor
+  int n_k;        // key rows per head
+  int nbq, nbk;   // ceil(n_q / 128), ceil(n_k / 128)
+  int heads_q;    // heads in the Q tensor
+  int heads_kv;   // heads in K / V / O
+  int n_units;    // work units
+  float scale_log2;  // softmax scale * log2(e)
+  const int32_t* work_list;  // unit -> hq * nbq + r (NULL: identity)
+  const int32_t* row_ptr;    // skip list (NULL: every key block)
+  const int32_t* col_idx;
+  int64_t nnz;
+  const int32_t* head_map;   // Q head -> K/V/O head (NULL: identity)
+  __nv_bfloat16* o;          // output [heads_kv][n_out][128]
+  float* lse;                // output [heads_kv][n_out] or NULL
+  int64_t n_out;             // rows per head of o / lse
+  // repeated heads: a packed anchor query q = f*(k*W) + j*W + c writes rows
+  // band_lo[j] .. band_hi[j]-1 of frame f, column c (rep_W = 0: off)
+  int rep_H, rep_W, rep_k;
+  int band_lo[kMaxAnchors], band_hi[kMaxAnchors];
+  // energy passes
+  float* lse_ws;       // [heads_q][nbq*128] row log2-sum-exp2 (log2 units)
+  float* energy;       // [heads_q][nbq][nbk] or NULL
+  int fuse_select;
+  long long eps_fx;    // eps in fixed point (50 fraction bits), rounded up
+  uint8_t* mask;
+  int32_t* kept;
+  uint16_t* counts;
+  int* status;         // device status word
+};
+
+struct AnchorTable {
+  int anchor[kMaxAnchors];
+};
+
+int launch_attention(int mode, const void* q, int q_rows, int q_heads, const void* k, const void* v, int kv_rows,
+                     int kv_heads, const KernelParams& p, cudaStream_t stream);
+
+long long eps_to_fixed(double eps);
+
+int launch_select(const float* energy, int64_t rows, int nb, long long eps_fx, uint8_t* mask, int32_t* kept,
+                  uint16_t* counts, cudaStream_t stream);
+int launch_accumulate(const uint8_t* mask, int64_t cells, uint16_t* counts, cudaStream_t stream);
+int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold, uint8_t* mask, int32_t* row_ptr,
+                     int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* row_cnt, int* status,
+                     cudaStream_t stream);
+int launch_gather(const void* q, int n, int heads, const int32_t* rep_heads, int n_rep, int H, int W, int k_anchor,
+                  const AnchorTable& tab, void* out, int* status, cudaStream_t stream);
+
+// Device address of the status word on the current device (NULL on failure).
+int* status_word();
+
+}  // namespace calibatt

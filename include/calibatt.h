@@ -1,0 +1,203 @@
+/*
+ * calibatt.h -- C ABI of libcalibatt, the B200 (sm_100a) hot path of
+ * CalibAtt (Calibrated Sparse Attention).
+ *
+ * Method: "Accelerating Text-to-Video Generation with Calibrated Sparse
+ * Attention" (Yehezkel et al., arXiv 2603.05503). Passages are cited by the
+ * zhichai.net explainer page of that paper ("explainer") and its sections:
+ *   §二  observations (B x B blocks with B = 128; repetition across rows),
+ *   §三  method: offline calibration (block energy, greedy eps selection,
+ *        rho aggregation, eps(t) schedule) and online inference (skip list
+ *        for non-repeated heads, k = 5 anchor rows for repeated heads),
+ *   §六  spatial repetition (row-major tokens within an H x W frame).
+ *
+ * Conventions (all entry points):
+ *  - Return value: CALIBATT_OK (0) or a negative calibatt_status code. Argument
+ *    errors are detected on the host before anything is enqueued; nothing is
+ *    launched when a call returns an error.
+ *  - Device pointers are caller-owned device memory; host pointers are marked
+ *    "host". The library never frees what it is given and keeps no pointer
+ *    after a call returns.
+ *  - Work is enqueued on the caller's stream (a cudaStream_t; NULL = legacy
+ *    default stream). No entry point synchronises except calibatt_get_status.
+ *  - Faults detected inside a kernel (a malformed skip list, a bounded wait
+ *    that ran out) are recorded in a device status word; read and clear it
+ *    with calibatt_get_status. Kernels never trap.
+ *  - Tensors are contiguous, row-major: q, k, v, o are bf16 [heads][n][128]
+ *    (d = 128 is the only supported head size), lse is fp32 [heads][n].
+ *    Device pointers to bf16 tensors must be 16-byte aligned.
+ *  - Blocks are B = 128 tokens of the flattened sequence (explainer §二):
+ *    nb = ceil(n / 128); a ragged last block is padded and masked.
+ *  - Token order: t = f*H*W + r*W + c (explainer §六).
+ */
+#ifndef CALIBATT_H_
+#define CALIBATT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t calibatt_bf16;          /* bf16 bit pattern */
+typedef struct CUstream_st* calibatt_stream_t; /* same handle as cudaStream_t */
+
+typedef enum calibatt_status {
+  CALIBATT_OK = 0,
+  CALIBATT_ERR_ARG = -1,         /* null pointer, bad size or count, short workspace */
+  CALIBATT_ERR_CSR = -2,         /* malformed skip list (row_ptr / col_idx) */
+  CALIBATT_ERR_ALIGN = -3,       /* device pointer not 16-byte aligned */
+  CALIBATT_ERR_UNSUPPORTED = -4, /* d != 128, or nb > 1024 for calibration */
+  CALIBATT_ERR_CUDA = -5,        /* a CUDA runtime/driver call failed */
+  CALIBATT_ERR_TIMEOUT = -6,     /* a bounded in-kernel wait ran out (device status) */
+  CALIBATT_ERR_CAPACITY = -7     /* nnz exceeds the caller's col_idx capacity */
+} calibatt_status;
+
+#define CALIBATT_BLOCK 128
+#define CALIBATT_HEAD_DIM 128
+#define CALIBATT_MAX_CALIB_NB 1024
+
+/* Text for a status code (static string, never NULL). */
+const char* calibatt_strerror(int code);
+
+/* Library ABI version (major*100 + minor). */
+int calibatt_version(void);
+
+/* Synchronises `stream`, then returns and clears the device status word
+ * (CALIBATT_OK if no kernel recorded a fault since the last call). */
+int calibatt_get_status(calibatt_stream_t stream);
+
+/* ---------------------------------------------------------------- host helpers */
+
+/* eps(t) = A + (C - A) * exp(-k t / T): the energy threshold schedule,
+ * C at the early high-noise step, relaxing towards A (explainer §三). */
+double calibatt_eps_schedule(double A, double C, double k, double t, double T);
+
+/* Checks a host copy of a skip list: row_ptr [heads*nb + 1] non-decreasing
+ * from 0 to nnz, every col_idx in [0, nb) and strictly ascending within a
+ * row. Returns CALIBATT_OK or CALIBATT_ERR_CSR (CALIBATT_ERR_ARG on bad sizes). */
+int calibatt_validate_csr(const int32_t* row_ptr, const int32_t* col_idx, int heads, int nb, int64_t nnz);
+
+/* Tile-scheduler plan (host): the work units (h*nb + r) of the heads marked
+ * active (all heads if head_active is NULL), sorted by kept-block count
+ * descending, ties by unit index (longest-processing-time order). Units with
+ * no kept block are included (their rows get O = 0, LSE = -inf).
+ * row_ptr: host [heads*nb + 1]; head_active: host [heads] or NULL;
+ * work_list: host output with room for heads*nb entries; *n_work: count. */
+int calibatt_build_plan(const int32_t* row_ptr, int heads, int nb, const uint8_t* head_active,
+                        int32_t* work_list, int32_t* n_work);
+
+/* Anchor rows of a repeated head: the centres of k equal bands of the H rows
+ * of a frame, a_j = floor((2j + 1) H / (2k)), j = 0..k-1 (explainer §三,
+ * "k = 5 anchor rows"; the pages do not fix the spacing, this is the plainest
+ * even one). anchors: host [k]. Requires 1 <= k <= H. */
+int calibatt_anchor_rows(int H, int k_anchor, int32_t* anchors);
+
+/* Integer form of "mean mask >= rho" for n inputs: the smallest count c in
+ * [0, n] with (double)c / n >= rho, or n + 1 if none (explainer §三). */
+int calibatt_rho_threshold(int n_inputs, double rho, int32_t* threshold);
+
+/* ---------------------------------------------------------------- inference */
+
+/* Block-sparse attention over a calibrated skip list (explainer §三, online
+ * inference for non-repeated heads; blocks of explainer §二).
+ * For each work unit u = h*nb + r in work_list[0..n_work): query rows
+ * [128r, min(128r+128, n)) of head h attend to the keys of the blocks
+ * col_idx[row_ptr[u] .. row_ptr[u+1]) (keys >= n masked):
+ *   O = softmax(scale * Q K^T) V,  lse = ln sum exp(scale * Q K^T).
+ * A unit with no kept block gets O = 0 and lse = -inf. Rows of heads that no
+ * unit names are not written.
+ *   q, k, v : device bf16 [heads][n][128];  o : device bf16 [heads][n][128]
+ *   row_ptr : device int32 [heads*nb + 1], global offsets into col_idx
+ *   col_idx : device int32 [nnz], ascending within a row, values in [0, nb)
+ *   work_list: device int32 [n_work] (from calibatt_build_plan)
+ *   lse     : device fp32 [heads][n] or NULL
+ * A malformed list is clamped in the kernel and reported as CALIBATT_ERR_CSR
+ * through calibatt_get_status; validate host copies with calibatt_validate_csr. */
+int calibatt_sparse_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v,
+                             int heads, int n, int d, float scale, const int32_t* row_ptr,
+                             const int32_t* col_idx, int64_t nnz, const int32_t* work_list, int32_t n_work,
+                             calibatt_bf16* o, float* lse, calibatt_stream_t stream);
+
+/* Workspace bytes needed by calibatt_repeat_attn_fwd (the packed anchor
+ * queries): n_rep * frames * k_anchor * W * 128 * 2, rounded up to 256. */
+size_t calibatt_repeat_workspace_size(int n_rep, int frames, int H, int W, int k_anchor);
+
+/* Spatially repeated heads (explainer §三 online inference for repeated heads,
+ * §六): for each head rep_heads[i], only the k anchor rows of every frame
+ * (calibatt_anchor_rows) are computed, as dense attention of those queries
+ * over all n = frames*H*W keys; every row r of a frame then receives, column
+ * by column, the output (and lse) of its nearest anchor row (ties -> lower
+ * anchor).
+ *   rep_heads: device int32 [n_rep], head indices in [0, heads)
+ *   ws       : device scratch of at least calibatt_repeat_workspace_size bytes
+ * Other heads' rows are not written. */
+int calibatt_repeat_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v,
+                             int heads, int frames, int H, int W, int d, int k_anchor, float scale,
+                             const int32_t* rep_heads, int32_t n_rep, calibatt_bf16* o, float* lse, void* ws,
+                             size_t ws_bytes, calibatt_stream_t stream);
+
+/* ---------------------------------------------------------------- calibration */
+
+/* Block energy of one calibration input (explainer §三 offline calibration,
+ * steps 1-2): with P = softmax(scale * Q K^T) over all n keys,
+ *   E[h][r][c] = (1 / |I_r|) * sum_{i in block r, j in block c} P_ij,
+ * |I_r| the query rows present in block r (128 except a ragged last block,
+ * which keeps every row sum at 1). P is never stored: a first pass writes the
+ * row log-sum-exp to lse_ws, a second recomputes S and reduces exp(S - lse)
+ * tile by tile.
+ * When fuse_select != 0 the same kernel applies the greedy selection of
+ * calibatt_select_mask at `eps` to each finished energy row and writes mask
+ * and/or kept and/or adds the mask into counts.
+ *   lse_ws : device fp32 scratch [heads][nb*128]
+ *   energy : device fp32 [heads][nb][nb] or NULL
+ *   mask   : device uint8 [heads][nb][nb] or NULL; kept: device int32 [heads][nb] or NULL
+ *   counts : device uint16 [heads][nb][nb] or NULL (counts += mask)
+ * Requires nb <= CALIBATT_MAX_CALIB_NB. */
+int calibatt_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int n, int d, float scale,
+                          float* lse_ws, float* energy, int fuse_select, double eps, uint8_t* mask,
+                          int32_t* kept, uint16_t* counts, calibatt_stream_t stream);
+
+/* Greedy eps selection (explainer §三, step 3) on rows of block energies:
+ * order the row's blocks by energy descending (equal energies: lower column
+ * first) and keep the shortest prefix whose running sum reaches eps. The sum
+ * is exact: each fp32 energy is taken in fixed point with 50 fraction bits
+ * (truncated), so the result does not depend on summation order. If no prefix
+ * reaches eps, every block with nonzero energy is kept; at least one block is
+ * always kept. Energies are clamped to [0, 4] (NaN -> 0).
+ *   energy : device fp32 [rows][nb], rows = heads*nb
+ *   mask   : device uint8 [rows][nb] or NULL; kept: device int32 [rows] or NULL
+ *   counts : device uint16 [rows][nb] or NULL (counts += mask)
+ * Requires nb <= CALIBATT_MAX_CALIB_NB. */
+int calibatt_select_mask(const float* energy, int heads, int nb, double eps, uint8_t* mask, int32_t* kept,
+                         uint16_t* counts, calibatt_stream_t stream);
+
+/* counts[i] += mask[i] (saturating at 65535) for `cells` entries: folds one
+ * calibration input's mask into the running sum over inputs (explainer §三). */
+int calibatt_accumulate_masks(const uint8_t* mask, int64_t cells, uint16_t* counts, calibatt_stream_t stream);
+
+/* Workspace bytes needed by calibatt_aggregate_masks. */
+size_t calibatt_aggregate_workspace_size(int heads, int nb);
+
+/* Aggregation and skip-list build (explainer §三): keep block (h, r, c) where
+ * counts / n_inputs >= rho (in integers: counts >= calibatt_rho_threshold),
+ * write the binary mask and its CSR skip list with global offsets, columns
+ * ascending.
+ *   counts  : device uint16 [heads][nb][nb]
+ *   mask    : device uint8 [heads][nb][nb] (output)
+ *   row_ptr : device int32 [heads*nb + 1] (output)
+ *   col_idx : device int32 [nnz_cap] (output)
+ *   nnz     : device int64 [1] (output: total kept blocks)
+ *   ws      : device scratch of calibatt_aggregate_workspace_size bytes
+ * If the kept total exceeds nnz_cap, col_idx holds the first nnz_cap entries
+ * and calibatt_get_status reports CALIBATT_ERR_CAPACITY. */
+int calibatt_aggregate_masks(const uint16_t* counts, int n_inputs, int heads, int nb, double rho, uint8_t* mask,
+                             int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, void* ws,
+                             size_t ws_bytes, calibatt_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CALIBATT_H_ */

@@ -1,0 +1,155 @@
+"""Host-side tests of libcalibatt (no GPU work is launched): the library
+loads, exports every entry point the header declares, its host helpers agree
+with the oracle, and argument errors are caught before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "calibatt.h")
+
+
+@pytest.fixture(scope="module")
+def binding():
+    from calibrated_block_sparse_b200 import binding as b, build
+    build.build()
+    b.load()
+    return b
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(calibatt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_north_star_calls():
+    names = _declared()
+    for n in ("calibatt_block_energy", "calibatt_select_mask", "calibatt_aggregate_masks",
+              "calibatt_sparse_attn_fwd", "calibatt_repeat_attn_fwd"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(binding):
+    lib = ctypes.CDLL(binding.library_path())
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_strerror_and_version(binding):
+    lib = binding.load()
+    assert lib.calibatt_version() >= 100
+    for code in range(0, -8, -1):
+        assert binding.strerror(code)
+    assert binding.strerror(-99) == "unknown status"
+
+
+def test_eps_schedule_matches_oracle(binding, oracle):
+    for t in (0, 10, 25, 49, 50):
+        assert binding.eps_schedule(0.84, 0.99, 5, t, 50) == pytest.approx(oracle.eps_schedule(0.84, 0.99, 5, t, 50),
+                                                                           abs=1e-15)
+    assert abs(binding.eps_schedule(0.84, 0.99, 5, 0.5, 1.0) - 0.852312749793585) < 1e-15
+
+
+@pytest.mark.parametrize("H,k", [(45, 5), (30, 5), (8, 5), (16, 16), (7, 1), (100, 64)])
+def test_anchor_rows_match_oracle(binding, oracle, H, k):
+    np.testing.assert_array_equal(binding.anchor_rows(H, k), oracle.anchor_rows(H, k))
+
+
+def test_rho_threshold_matches_oracle_decisions(binding, oracle):
+    for n in (1, 2, 3, 8, 10, 16, 64):
+        for rho in (0.0, 0.1, 0.3, 0.5, 0.7, 1 / 3, 0.9999, 1.0, 1.5):
+            thr = binding.rho_threshold(n, rho)
+            counts = np.arange(n + 1, dtype=np.int32)
+            ref = oracle.binarize_counts(counts, n, rho)
+            np.testing.assert_array_equal((counts >= thr).astype(np.uint8), ref)
+
+
+def test_validate_csr(binding, oracle):
+    rng = np.random.default_rng(1)
+    mask = (rng.random((2, 9, 9)) < 0.4).astype(np.uint8)
+    rp, ci = oracle.mask_to_csr(mask)
+    assert binding.validate_csr(rp, ci, 2, 9) == 0
+    bad = ci.copy()
+    bad[0] = 9
+    assert binding.validate_csr(rp, bad, 2, 9) == -2
+    if ci.size > 1 and rp[1] - rp[0] > 1:
+        dup = ci.copy()
+        dup[1] = dup[0]
+        assert binding.validate_csr(rp, dup, 2, 9) == -2
+    rp2 = rp.copy()
+    rp2[3] = rp2[4] + 1
+    assert binding.validate_csr(rp2, ci, 2, 9) == -2
+
+
+def test_build_plan_is_longest_first(binding, oracle):
+    rng = np.random.default_rng(2)
+    mask = (rng.random((3, 7, 7)) < rng.random((3, 1, 1))).astype(np.uint8)
+    rp, _ = oracle.mask_to_csr(mask)
+    work = binding.build_plan(rp, 3, 7)
+    nnz = np.diff(rp)
+    assert sorted(work.tolist()) == list(range(21))
+    assert np.all(np.diff(nnz[work]) <= 0)
+    # ties keep unit order
+    for a, b in zip(work, work[1:]):
+        if nnz[a] == nnz[b]:
+            assert a < b
+    work = binding.build_plan(rp, 3, 7, head_active=np.array([0, 1, 0], np.uint8))
+    assert sorted(work.tolist()) == list(range(7, 14))
+
+
+def test_argument_errors_are_caught_on_the_host(binding):
+    lib = binding.load()
+    P = ctypes.c_void_p
+    fake = P(0x100000)       # aligned, never dereferenced: calls must fail first
+    odd = P(0x100008)        # 8-byte aligned only
+    # head dim other than 128
+    assert lib.calibatt_sparse_attn_fwd(fake, fake, fake, 1, 256, 64, 0.1, fake, fake, 4, fake, 2, fake, None,
+                                        None) == -4
+    # misaligned q
+    assert lib.calibatt_sparse_attn_fwd(odd, fake, fake, 1, 256, 128, 0.1, fake, fake, 4, fake, 2, fake, None,
+                                        None) == -3
+    # non-positive scale, missing row_ptr, bad sizes
+    assert lib.calibatt_sparse_attn_fwd(fake, fake, fake, 1, 256, 128, 0.0, fake, fake, 4, fake, 2, fake, None,
+                                        None) == -1
+    assert lib.calibatt_sparse_attn_fwd(fake, fake, fake, 1, 256, 128, 0.1, None, fake, 4, fake, 2, fake, None,
+                                        None) == -1
+    assert lib.calibatt_sparse_attn_fwd(fake, fake, fake, 0, 256, 128, 0.1, fake, fake, 4, fake, 2, fake, None,
+                                        None) == -1
+    assert lib.calibatt_sparse_attn_fwd(fake, fake, fake, 1, 256, 128, 0.1, fake, fake, 4, fake, 3, fake, None,
+                                        None) == -1
+    # repeat: k larger than H, workspace too small, too many anchors
+    assert lib.calibatt_repeat_attn_fwd(fake, fake, fake, 2, 2, 4, 8, 128, 5, 0.1, fake, 1, fake, None, fake,
+                                        1 << 30, None) == -1
+    assert lib.calibatt_repeat_attn_fwd(fake, fake, fake, 2, 2, 8, 8, 128, 5, 0.1, fake, 1, fake, None, fake,
+                                        16, None) == -1
+    assert lib.calibatt_repeat_attn_fwd(fake, fake, fake, 2, 2, 80, 8, 128, 70, 0.1, fake, 1, fake, None, fake,
+                                        1 << 30, None) == -4
+    # calibration beyond 1024 blocks per row
+    assert lib.calibatt_block_energy(fake, fake, 1, 1025 * 128, 128, 0.1, fake, None, 0, 0.0, None, None, None,
+                                     None) == -4
+    assert lib.calibatt_select_mask(fake, 1, 2000, 0.9, fake, None, None, None) == -4
+    assert lib.calibatt_select_mask(fake, 1, 16, 0.9, None, None, None, None) == -1
+    assert lib.calibatt_select_mask(fake, 1, 16, float("nan"), fake, None, None, None) == -1
+    # aggregation: short workspace, zero inputs
+    assert lib.calibatt_aggregate_masks(fake, 4, 1, 16, 0.5, fake, fake, fake, 256, fake, fake, 4, None) == -1
+    assert lib.calibatt_aggregate_masks(fake, 0, 1, 16, 0.5, fake, fake, fake, 256, fake, fake, 1024, None) == -1
+    assert lib.calibatt_accumulate_masks(None, 10, fake, None) == -1
+
+
+def test_workspace_sizes(binding):
+    lib = binding.load()
+    assert binding.repeat_workspace_size(8, 21, 45, 80, 5) == 8 * 21 * 5 * 80 * 256
+    assert lib.calibatt_aggregate_workspace_size(40, 591) >= 40 * 591 * 4
+    assert lib.calibatt_aggregate_workspace_size(0, 5) == 0
+
+
+def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
+    from calibrated_block_sparse_b200 import binding as b
+    monkeypatch.setattr(b, "_lib", None)
+    monkeypatch.setattr(b, "library_path", lambda: str(tmp_path / "absent.so"))
+    with pytest.raises(ImportError):
+        b.load()

@@ -1,0 +1,148 @@
+"""GPU parity: block-sparse and repeated-head attention through the C ABI,
+element by element against the fp64 oracle on the same bf16 inputs.
+
+Tolerance (stated by the method's parity rule for bf16 inputs with fp32
+accumulation): max|O - O_ref| <= 1e-2 * max|O_ref| + 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from calibrated_block_sparse_b200 import synth
+from gpu_util import attn_tolerance_ok, bf16_to_f64, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_sparse(binding, q, k, v, mask):
+    import oracle
+    heads, nb, _ = mask.shape
+    row_ptr, col_idx = oracle.mask_to_csr(mask)  # the reference skip list
+    assert binding.validate_csr(row_ptr, col_idx, heads, nb) == 0
+    work = binding.build_plan(row_ptr, heads, nb)
+    dev = torch.device("cuda")
+    o, lse = binding.sparse_attn_fwd(q.to(dev), k.to(dev), v.to(dev), torch.from_numpy(row_ptr).to(dev),
+                                     torch.from_numpy(col_idx).to(dev), torch.from_numpy(work).to(dev))
+    assert binding.get_status() == 0
+    return bf16_to_f64(o), lse.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("heads,n,keep,seed", [
+    (1, 2048, 0.4, 1),     # the tiny workload's shape: 16 blocks
+    (2, 300, 0.6, 2),      # ragged: last block 44 rows
+    (3, 1000, 0.3, 3),     # ragged: last block 104 rows, several tiles per CTA slot
+    (2, 128, 1.0, 4),      # a single block
+    (1, 4096 + 80, 0.25, 5),  # 33 blocks, last 80 rows (Wan-720p's tail)
+])
+def test_sparse_attention_matches_oracle(oracle, heads, n, keep, seed):
+    binding = require_gpu()
+    q, k, v = synth.plain_qkv(heads, n, seed=seed, std=1.5)
+    nb = (n + 127) // 128
+    mask = synth.random_mask(heads, nb, keep, seed=seed)
+    o, lse = _run_sparse(binding, q, k, v, mask)
+    o_ref, lse_ref = oracle.masked_attention(synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v), mask)
+    ok, err, bound = attn_tolerance_ok(o, o_ref)
+    assert ok, (err, bound)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=2e-3)
+
+
+def test_all_ones_mask_is_dense_attention(oracle):
+    binding = require_gpu()
+    q, k, v = synth.plain_qkv(2, 700, seed=7)
+    nb = 6
+    o, lse = _run_sparse(binding, q, k, v, np.ones((2, nb, nb), np.uint8))
+    o_ref, _ = oracle.masked_attention(synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v),
+                                       np.ones((2, nb, nb), np.uint8))
+    assert attn_tolerance_ok(o, o_ref)[0]
+
+
+def test_empty_rows_and_large_scores(oracle):
+    binding = require_gpu()
+    # large-magnitude scores exercise the running-max rescale; an empty row
+    # must come out as O = 0, lse = -inf
+    q, k, v = synth.plain_qkv(1, 640, seed=8, std=4.0)
+    mask = synth.random_mask(1, 5, 0.5, seed=8)
+    mask[0, 2] = 0
+    o, lse = _run_sparse(binding, q, k, v, mask)
+    o_ref, lse_ref = oracle.masked_attention(synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v), mask)
+    assert attn_tolerance_ok(o, o_ref)[0]
+    assert np.all(o[0, 256:384] == 0) and np.all(np.isneginf(lse[0, 256:384]))
+
+
+def test_rows_of_other_heads_untouched():
+    binding = require_gpu()
+    import oracle
+    q, k, v = synth.plain_qkv(3, 256, seed=9)
+    mask = np.ones((3, 2, 2), np.uint8)
+    row_ptr, col_idx = oracle.mask_to_csr(mask)
+    work = binding.build_plan(row_ptr, 3, 2, head_active=np.array([1, 0, 1], np.uint8))
+    assert len(work) == 4
+    dev = torch.device("cuda")
+    o = torch.full((3, 256, 128), 7.0, dtype=torch.bfloat16, device=dev)
+    binding.sparse_attn_fwd(q.to(dev), k.to(dev), v.to(dev), torch.from_numpy(row_ptr).to(dev),
+                            torch.from_numpy(col_idx).to(dev), torch.from_numpy(work).to(dev), o=o)
+    assert binding.get_status() == 0
+    assert torch.all(o[1] == 7.0)
+    assert not torch.any(o[0] == 7.0)
+
+
+@pytest.mark.parametrize("F,H,W,kk", [(3, 8, 16, 5), (2, 6, 20, 6), (2, 30, 5, 5), (4, 5, 9, 2)])
+def test_repeat_attention_matches_oracle(oracle, F, H, W, kk):
+    binding = require_gpu()
+    heads = 3
+    n = F * H * W
+    q, k, v = synth.plain_qkv(heads, n, seed=10 + H)
+    rep = [0, 2]
+    dev = torch.device("cuda")
+    o = torch.zeros((heads, n, 128), dtype=torch.bfloat16, device=dev)
+    o, lse = binding.repeat_attn_fwd(q.to(dev), k.to(dev), v.to(dev), F, H, W,
+                                     torch.tensor(rep, dtype=torch.int32, device=dev), k_anchor=kk, o=o)
+    assert binding.get_status() == 0
+    o_ref, lse_ref = oracle.repeat_attention(synth.bf16_bits(q[rep]), synth.bf16_bits(k[rep]),
+                                             synth.bf16_bits(v[rep]), F, H, W, k_anchor=kk)
+    og = bf16_to_f64(o)
+    ok, err, bound = attn_tolerance_ok(og[rep], o_ref)
+    assert ok, (err, bound)
+    np.testing.assert_allclose(lse.cpu().numpy()[rep], lse_ref, rtol=0, atol=2e-3)
+    assert np.all(og[1] == 0)  # not a repeat head: untouched
+    # rows of one band are exact copies of their anchor row
+    a = binding.anchor_rows(H, kk)
+    for f in range(F):
+        for r in range(H):
+            j = int(np.argmin(np.abs(r - a)))
+            src = f * H * W + int(a[j]) * W
+            dst = f * H * W + r * W
+            assert np.array_equal(og[rep, dst:dst + W], og[rep, src:src + W])
+
+
+def test_repeat_with_every_row_an_anchor_is_plain_attention(oracle):
+    binding = require_gpu()
+    F, H, W = 2, 8, 24
+    n = F * H * W
+    q, k, v = synth.plain_qkv(1, n, seed=12)
+    dev = torch.device("cuda")
+    o, _ = binding.repeat_attn_fwd(q.to(dev), k.to(dev), v.to(dev), F, H, W,
+                                   torch.zeros(1, dtype=torch.int32, device=dev), k_anchor=H)
+    nb = (n + 127) // 128
+    o_ref, _ = oracle.masked_attention(synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v),
+                                       np.ones((1, nb, nb), np.uint8))
+    assert attn_tolerance_ok(bf16_to_f64(o), o_ref)[0]
+
+
+def test_malformed_skip_list_is_reported_not_faulted():
+    binding = require_gpu()
+    import oracle
+    q, k, v = synth.plain_qkv(1, 256, seed=13)
+    mask = np.ones((1, 2, 2), np.uint8)
+    row_ptr, col_idx = oracle.mask_to_csr(mask)
+    bad = col_idx.copy()
+    bad[1] = 57  # column out of range
+    assert binding.validate_csr(row_ptr, bad, 1, 2) != 0
+    dev = torch.device("cuda")
+    binding.get_status()
+    binding.sparse_attn_fwd(q.to(dev), k.to(dev), v.to(dev), torch.from_numpy(row_ptr).to(dev),
+                            torch.from_numpy(bad).to(dev), torch.tensor([0, 1], dtype=torch.int32, device=dev))
+    assert binding.get_status() == -2  # CALIBATT_ERR_CSR
+    assert binding.get_status() == 0   # cleared
