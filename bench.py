@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Benchmark of the CalibAtt hot path on B200 (one JSON line on rank 0).
+
+One step = one attention call of the Wan 2.1 14B 720p shape (40 heads,
+N = 75600 = 21 x 45 x 80 tokens, d = 128, bf16): block-sparse attention of the
+32 non-repeated heads over their skip lists (random per-head masks, 62.5 %
+mean block sparsity) followed by the anchor-row attention of the 8 repeated
+heads (k = 5 anchor rows of 45). The metric is kept-tile attention TFLOPS
+(algorithmic: 4 * d * valid query rows * valid key columns per kept tile),
+reported against the BF16 tensor roofline and next to the same kernel run at
+0 % sparsity. The calibration kernels (block energy with fused selection,
+standalone selection, aggregation) are timed in the same run on the same
+shape and reported under "calibration".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun), every rank runs its own copy of the workload on its own
+inputs (weak scaling, no data-path collective); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from calibrated_block_sparse_b200 import synth  # noqa: E402
+
+D = 128
+METRIC = "kept-tile attention TFLOPS"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- work accounting
+
+def valid_sizes(n, nb):
+    v = np.full(nb, 128, np.int64)
+    v[-1] = n - (nb - 1) * 128
+    return v
+
+
+def sparse_flops(mask, heads, n):
+    """Algorithmic flops of the block-sparse heads: 4 d |valid q| |valid k| per kept tile."""
+    nb = mask.shape[-1]
+    v = valid_sizes(n, nb)
+    pair = np.outer(v, v)
+    return float(4 * D * sum(int((mask[h].astype(np.int64) * pair).sum()) for h in heads))
+
+
+def repeat_flops(wl, n_rep):
+    return float(4 * D * wl.F * wl.k_anchor * wl.W * wl.n * n_rep)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif args.impl == "ours":
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU baseline (oracle)
+
+def cpu_oracle_sample(wl, q_cpu, k_cpu, v_cpu, heads, masks, budget_s, rng, repeat=False):
+    """Time the fp64 oracle on randomly sampled query rows of the given heads.
+
+    Returns (seconds, algorithmic flops, rows, threads)."""
+    import oracle
+    threads = os.cpu_count() or 1
+    nb = wl.nb
+    v_sz = valid_sizes(wl.n, nb)
+    spent, flops, rows_done, batch = 0.0, 0.0, 0, max(threads, 8)
+    while spent < budget_s:
+        hi = int(rng.integers(len(heads)))
+        rows = rng.integers(0, wl.n, size=batch).astype(np.int64)
+        qb, kb, vb = (synth.bf16_bits(t[hi:hi + 1]) for t in (q_cpu, k_cpu, v_cpu))
+        t0 = time.perf_counter()
+        if repeat:
+            oracle.repeat_attention(qb, kb, vb, wl.F, wl.H, wl.W, wl.k_anchor, rows=rows, threads=threads)
+            flops += 4.0 * D * wl.n * batch
+        else:
+            oracle.masked_attention(qb, kb, vb, masks[heads[hi]][None], rows=rows, threads=threads)
+            kept = masks[heads[hi]][rows // 128].astype(np.int64) @ v_sz
+            flops += 4.0 * D * float(kept.sum())
+        spent += time.perf_counter() - t0
+        rows_done += batch
+    return spent, flops, rows_done, threads
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the oracle as it stands, on the host cores, same metric."""
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    masks = synth.random_block_masks(wl) if wl.repeat_heads or args.workload == "wan720" else \
+        np.ones((wl.heads, wl.nb, wl.nb), np.uint8)
+    sparse_heads = [h for h in range(wl.heads) if h not in wl.repeat_heads]
+    rng = np.random.default_rng(1234)
+    hs = [sparse_heads[0]]
+    q, k, v = synth.qkv(wl, 0, heads=hs)
+    qm = np.stack([masks[h] for h in hs])
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, q, k, v, [0], qm, 0.2, rng)
+    tot_s, tot_f, rows, threads = 0.0, 0.0, 0, 1
+    for _ in range(args.steps):
+        s, f, r, threads = cpu_oracle_sample(wl, q, k, v, [0], qm, per_step, rng)
+        tot_s += s
+        tot_f += f
+        rows += r
+    value = tot_f / tot_s / 1e12
+    sample = (f"{rows} query rows of one block-sparse head of {wl.name}, fp64 oracle "
+              f"(plain C, {threads} threads), throughput in kept-tile flops")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "heads": wl.heads, "n": wl.n, "d": D},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def cuda_time(fn, reps, stream):
+    """Average device ms of fn() over reps, CUDA events on `stream`."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(reps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / reps
+
+
+def run_ours(args, world, rank, local):
+    from calibrated_block_sparse_b200 import binding
+    binding.load()
+    wl = synth.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    n, nb, heads = wl.n, wl.nb, wl.heads
+    rep_heads = list(wl.repeat_heads)
+    sparse_heads = [h for h in range(heads) if h not in rep_heads]
+
+    # inputs: resident in HBM before the timed region
+    q, k, v = synth.qkv(wl, 1000 + rank, device=dev)
+    if args.workload == "wan720":
+        masks = synth.random_block_masks(wl)
+    else:
+        masks = (np.random.default_rng(7).random((heads, nb, nb)) < 0.32).astype(np.uint8)
+        masks[:, np.arange(nb), np.arange(nb)] = 1
+    # skip lists built on the GPU by the aggregation kernel (one input, rho 0.5)
+    counts = torch.from_numpy(masks.astype(np.int16)).to(dev).view(torch.uint16)
+    mask_d, row_ptr, col_idx, _ = binding.aggregate_masks(counts, 1, 0.5)
+    binding.check_status(what="aggregate_masks")
+    row_ptr_h = row_ptr.cpu().numpy()
+    head_active = np.array([h not in rep_heads for h in range(heads)], np.uint8)
+    work = torch.from_numpy(binding.build_plan(row_ptr_h, heads, nb, head_active)).to(dev)
+    rep_t = torch.tensor(rep_heads, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((heads, n), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(binding.repeat_workspace_size(max(len(rep_heads), 1), wl.F, wl.H, wl.W, wl.k_anchor), 256),
+                     dtype=torch.uint8, device=dev)
+
+    f_sparse = sparse_flops(masks, sparse_heads, n)
+    f_rep = repeat_flops(wl, len(rep_heads))
+    f_step = f_sparse + f_rep
+    kept_frac = float(np.mean([masks[h].mean() for h in sparse_heads]))
+
+    def sparse_call():
+        binding.sparse_attn_fwd(q, k, v, row_ptr, col_idx, work, o=o, lse=lse, stream=stream)
+
+    def repeat_call():
+        if rep_heads:
+            binding.repeat_attn_fwd(q, k, v, wl.F, wl.H, wl.W, rep_t, wl.k_anchor, o=o, lse=lse, ws=ws,
+                                    stream=stream)
+
+    def step():
+        sparse_call()
+        repeat_call()
+
+    launches_per_step = 1 + (2 if rep_heads else 0)
+    for _ in range(args.warmup):
+        step()
+    binding.check_status(what="warmup")
+
+    # ---- timed region: K steps, events per step around the sparse kernel
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t_start.record(stream)
+        for e0, e1, e2 in evs:
+            e0.record(stream)
+            sparse_call()
+            e1.record(stream)
+            repeat_call()
+            e2.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    binding.check_status(what="timed steps")
+    sparse_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs) / args.steps
+    repeat_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in evs) / args.steps
+    ms_step = elapsed_ms / args.steps
+    value = world * f_step / (ms_step * 1e-3) / 1e12
+
+    # ---- 0 %-sparse run: the same kernel with every block kept, all 40 heads
+    full = torch.ones((heads, nb, nb), dtype=torch.int16, device=dev).view(torch.uint16)
+    _, rp_full, ci_full, _ = binding.aggregate_masks(full, 1, 0.5)
+    work_full = torch.from_numpy(binding.build_plan(rp_full.cpu().numpy(), heads, nb)).to(dev)
+
+    def dense_call():
+        binding.sparse_attn_fwd(q, k, v, rp_full, ci_full, work_full, o=o, lse=lse, stream=stream)
+
+    dense_call()
+    dense_ms = cuda_time(dense_call, max(2, min(5, args.steps)), stream)
+    binding.check_status(what="dense")
+    f_dense = float(4 * D * n * n * heads)
+    del rp_full, ci_full, work_full, full
+
+    # ---- end to end through the C ABI with host buffers: H2D q,k,v, call, D2H o
+    e2e = None
+    if not args.no_e2e:
+        qh = q.cpu().pin_memory()
+        kh = k.cpu().pin_memory()
+        vh = v.cpu().pin_memory()
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(o, non_blocking=True)
+
+        e2e_step()
+        reps = max(2, min(5, args.steps))
+        barrier(world)
+        e2e_ms = max_over_ranks(cuda_time(e2e_step, reps, stream), world)
+        binding.check_status(what="e2e")
+        e2e = {"value": world * f_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()),
+               "d2h_bytes_per_step": int(o.numel() * o.element_size()), "ms_per_step": e2e_ms}
+        del qh, kh, vh, oh
+
+    # ---- calibration kernels on the same shape (8 heads of it)
+    calib = None
+    if not args.no_calib:
+        ch = 8
+        qc, kc = q[:ch].contiguous(), k[:ch].contiguous()
+        lse_ws = torch.empty((ch, nb * 128), dtype=torch.float32, device=dev)
+        energy = torch.empty((ch, nb, nb), dtype=torch.float32, device=dev)
+        cmask = torch.empty((ch, nb, nb), dtype=torch.uint8, device=dev)
+        ccounts = torch.zeros((ch, nb, nb), dtype=torch.uint16, device=dev)
+
+        def energy_call():
+            binding.block_energy(qc, kc, eps=0.9, energy=energy, mask=cmask, counts=ccounts, lse_ws=lse_ws,
+                                 stream=stream)
+
+        energy_call()
+        e_ms = cuda_time(energy_call, 2, stream)
+        f_energy_alg = float(2 * D * n * n * ch)  # one S = Q K^T per input
+        f_energy_issued = 2 * f_energy_alg        # two passes recompute S
+
+        def select_call():
+            binding.select_mask(energy, 0.9, mask=cmask, kept=False, stream=stream)
+
+        select_call()
+        s_ms = cuda_time(select_call, 5, stream)
+        sel_bytes = ch * nb * nb * (4 + 1)
+        agg_ws = torch.empty(binding.load().calibatt_aggregate_workspace_size(ch, nb), dtype=torch.uint8, device=dev)
+        am = torch.empty((ch, nb, nb), dtype=torch.uint8, device=dev)
+        arp = torch.empty(ch * nb + 1, dtype=torch.int32, device=dev)
+        aci = torch.empty(ch * nb * nb, dtype=torch.int32, device=dev)
+        annz = torch.zeros(1, dtype=torch.int64, device=dev)
+        lib = binding.load()
+
+        def agg_call():
+            lib.calibatt_aggregate_masks(binding._ptr(ccounts), 64, ch, nb, 0.5, binding._ptr(am),
+                                         binding._ptr(arp), binding._ptr(aci), aci.numel(), binding._ptr(annz),
+                                         binding._ptr(agg_ws), agg_ws.numel(), binding._stream(stream))
+
+        agg_call()
+        a_ms = cuda_time(agg_call, 5, stream)
+        binding.check_status(what="calibration")
+        kept_agg = int(annz.item())
+        agg_bytes = ch * nb * nb * (2 + 1 + 1) + kept_agg * 4 + (ch * nb + 1) * 4 * 3
+        calib = {
+            "shape": f"{ch} heads x N={n}",
+            "energy_ms": e_ms, "energy_tflops_algorithmic": f_energy_alg / (e_ms * 1e-3) / 1e12,
+            "energy_tflops_issued": f_energy_issued / (e_ms * 1e-3) / 1e12,
+            "select_ms": s_ms, "select_gbs": sel_bytes / (s_ms * 1e-3) / 1e9,
+            "aggregate_ms": a_ms, "aggregate_gbs": agg_bytes / (a_ms * 1e-3) / 1e9,
+            "eps": 0.9, "kept_fraction_at_eps": float(cmask.float().mean().item()),
+        }
+        del qc, kc, lse_ws, energy, cmask, ccounts
+
+    # ---- roofline of the dominant kernel (the block-sparse attention kernel)
+    pk, pk_src = peaks()
+    long_run = elapsed_ms > 1000.0
+    peak = pk.get("bf16_tflops_sustained" if long_run else "bf16_tflops")
+    achieved = f_sparse / (sparse_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attn_kernel<attention> (block-sparse heads)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{pk_src} {'sustained' if long_run else 'burst'} bf16",
+                "traffic": args.traffic_bytes}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        hs = [sparse_heads[0]]
+        qc, kc, vc = (t[hs].cpu() for t in (q, k, v))
+        s, f, rows, threads = cpu_oracle_sample(wl, qc, kc, vc, [0], np.stack([masks[h] for h in hs]),
+                                                args.cpu_seconds, np.random.default_rng(5))
+        cpu = {"value": f / s / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{rows} query rows of one block-sparse head, fp64 plain-C oracle, {s:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {heads} heads x N={n} (F={wl.F},H={wl.H},W={wl.W}), d={D}, "
+                                   f"{len(sparse_heads)} block-sparse + {len(rep_heads)} repeated (k={wl.k_anchor})",
+                       "kept_block_fraction": kept_frac, "block_sparsity": 1 - kept_frac,
+                       "l2": "inputs (3 x %.2f GB) larger than L2; no flush" % (q.numel() * 2 / 1e9),
+                       "parallelism": f"replica per GPU x{world}"},
+            "gpu_launches": launches_per_step * args.steps,
+            "sparse_ms": sparse_ms, "repeat_ms": repeat_ms,
+            "dense_ms": dense_ms, "dense_tflops": f_dense / (dense_ms * 1e-3) / 1e12,
+            "speedup_vs_dense": dense_ms / ms_step,
+            "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "calibration": calib,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["wan720", "wan480", "mochi480"], default="wan720")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-calib", action="store_true")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="dram bytes per launch of the sparse kernel from an ncu capture")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

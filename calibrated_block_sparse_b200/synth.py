@@ -94,22 +94,26 @@ def fourier_features(wl: Workload, head: int) -> torch.Tensor:
     return out
 
 
-def _normal(shape, seed: int) -> torch.Tensor:
-    g = torch.Generator(device="cpu")
+def _normal(shape, seed: int, device="cpu") -> torch.Tensor:
+    g = torch.Generator(device=device)
     g.manual_seed(seed)
-    return torch.randn(shape, generator=g, dtype=torch.float32)
+    return torch.randn(shape, generator=g, dtype=torch.float32, device=device)
 
 
-def qkv(wl: Workload, input_idx: int, heads=None, with_v: bool = True):
-    """bf16 CPU tensors q, k (and v), [len(heads)][n][128] for one input."""
+def qkv(wl: Workload, input_idx: int, heads=None, with_v: bool = True, device="cpu"):
+    """bf16 tensors q, k (and v), [len(heads)][n][128] for one input.
+
+    The random stream depends on the device's generator: CPU generation is the
+    reference recipe (used for oracle parity); generation on a CUDA device is a
+    faster stand-in with the same distribution (benchmark inputs)."""
     heads = list(range(wl.heads)) if heads is None else list(heads)
     qs, ks, vs = [], [], []
     for h in heads:
-        e = fourier_features(wl, h)
-        qs.append((_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 1)) + 2.0 * e).to(torch.bfloat16))
-        ks.append((_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 2)) + 2.0 * e).to(torch.bfloat16))
+        e = fourier_features(wl, h).to(device)
+        qs.append((_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 1), device) + 2.0 * e).to(torch.bfloat16))
+        ks.append((_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 2), device) + 2.0 * e).to(torch.bfloat16))
         if with_v:
-            vs.append(_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 3)).to(torch.bfloat16))
+            vs.append(_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 3), device).to(torch.bfloat16))
     q = torch.stack(qs)
     k = torch.stack(ks)
     v = torch.stack(vs) if with_v else None
