@@ -66,6 +66,7 @@ def load(build_if_missing: bool = False):
             "calibatt_accumulate_masks": (i32, [P, i64, P, P]),
             "calibatt_aggregate_workspace_size": (sz, [i32, i32]),
             "calibatt_aggregate_masks": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P, sz, P]),
+            "calibatt_aggregate_masks_noalloc": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -282,4 +283,16 @@ def aggregate_masks(counts, n_inputs, rho=0.5, nnz_cap=None, ws=None, stream=Non
     if trim:
         total = int(nnz.item())
         col_idx = col_idx[:total]
+    return mask, row_ptr, col_idx, nnz
+
+
+def aggregate_masks_noalloc(counts, n_inputs, rho, mask, row_ptr, col_idx, nnz, stream=None):
+    """calibatt_aggregate_masks_noalloc: the caller passes every output buffer and
+    the library allocates nothing (its scratch is a static device array)."""
+    _cuda_tensor(counts, torch.uint16, "counts")
+    heads, nb, _ = counts.shape
+    rc = load().calibatt_aggregate_masks_noalloc(_ptr(counts), int(n_inputs), heads, nb, float(rho), _ptr(mask),
+                                                 _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(nnz),
+                                                 _stream(stream))
+    _check(rc, "calibatt_aggregate_masks_noalloc")
     return mask, row_ptr, col_idx, nnz

@@ -196,6 +196,32 @@ int calibatt_aggregate_masks(const uint16_t* counts, int n_inputs, int heads, in
                              int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, void* ws,
                              size_t ws_bytes, calibatt_stream_t stream);
 
+/* ---------------------------------------------------------------- no-allocation variant */
+
+/* Largest heads * nb accepted by calibatt_aggregate_masks_noalloc. */
+#define CALIBATT_NOALLOC_MAX_ROWS (1 << 18)
+
+/* calibatt_aggregate_masks without a workspace argument. The method has no
+ * counterpart for this: it exists for callers that cannot allocate device
+ * memory when they build a skip list -- for example a plugin that only
+ * receives pointers from a host engine whose allocator owns the GPU's memory,
+ * or a serving loop under a fixed memory budget where an allocation could fail
+ * or stall. Same arguments, outputs and errors as calibatt_aggregate_masks
+ * (the caller still passes counts, mask, row_ptr, col_idx and nnz); the
+ * per-row counts live in a static device array of CALIBATT_NOALLOC_MAX_ROWS
+ * int32 (1 MiB), held by every GPU that loads the library until exit.
+ *  - Returns CALIBATT_ERR_ARG when heads * nb > CALIBATT_NOALLOC_MAX_ROWS.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the array: calls whose kernels overlap on the GPU (for
+ *    example on two streams at once) race and corrupt each other's results.
+ *    Every row count is rewritten by each call, so nothing needs clearing. */
+int calibatt_aggregate_masks_noalloc(const uint16_t* counts, int n_inputs, int heads, int nb, double rho,
+                                     uint8_t* mask, int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap,
+                                     int64_t* nnz, calibatt_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
