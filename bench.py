@@ -238,6 +238,10 @@ def run_ours(args, world, rank, local):
     from calibrated_block_sparse_b200 import binding
     binding.load()
     wl = synth.WORKLOADS[args.workload]
+    if args.heads:
+        # a smaller case of the same kernels: the first `heads` heads only
+        import dataclasses
+        wl = dataclasses.replace(wl, heads=args.heads, repeat_heads=tuple(h for h in wl.repeat_heads if h < args.heads))
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     n, nb, heads = wl.n, wl.nb, wl.heads
@@ -247,7 +251,7 @@ def run_ours(args, world, rank, local):
     # inputs: resident in HBM before the timed region
     q, k, v = synth.qkv(wl, 1000 + rank, device=dev)
     if args.workload == "wan720":
-        masks = synth.random_block_masks(wl)
+        masks = synth.random_block_masks(synth.WORKLOADS["wan720"])[:heads]
     else:
         masks = (np.random.default_rng(7).random((heads, nb, nb)) < 0.32).astype(np.uint8)
         masks[:, np.arange(nb), np.arange(nb)] = 1
@@ -354,7 +358,7 @@ def run_ours(args, world, rank, local):
     # ---- calibration kernels on the same shape (8 heads of it)
     calib = None
     if not args.no_calib:
-        ch = 8
+        ch = min(8, heads)
         qc, kc = q[:ch].contiguous(), k[:ch].contiguous()
         lse_ws = torch.empty((ch, nb * 128), dtype=torch.float32, device=dev)
         energy = torch.empty((ch, nb, nb), dtype=torch.float32, device=dev)
@@ -451,6 +455,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["wan720", "wan480", "mochi480"], default="wan720")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--heads", type=int, default=0, help="run only the first HEADS heads (profiling case)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-calib", action="store_true")
     ap.add_argument("--traffic-bytes", type=float, default=None,

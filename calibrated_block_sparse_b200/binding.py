@@ -32,7 +32,8 @@ class CalibattError(RuntimeError):
 
 
 def library_path() -> str:
-    return _build.LIB
+    """Path of libcalibatt.so: CALIBATT_LIBRARY if set, else the in-tree build."""
+    return os.environ.get("CALIBATT_LIBRARY") or _build.LIB
 
 
 def load(build_if_missing: bool = False):

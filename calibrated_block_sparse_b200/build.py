@@ -39,14 +39,18 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, jobs: int = 4) -> str:
-    if not force and not needs_build():
+def build(force: bool = False, ptxas_verbose: bool = False, jobs: int = 4, out_path: str = None,
+          defines=()) -> str:
+    """Compile every csrc/*.cu and link libcalibatt.so (in-tree unless out_path)."""
+    target = out_path or LIB
+    if not force and not defines and out_path is None and not needs_build():
         return LIB
     cc = nvcc()
     flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
                     "--expt-relaxed-constexpr"]
     if ptxas_verbose:
         flags += ["-Xptxas", "-v"]
+    flags += [f"-D{d}" for d in defines]
     with tempfile.TemporaryDirectory(prefix="calibatt_build_") as tmp:
         objs = []
         procs = []
@@ -60,11 +64,11 @@ def build(force: bool = False, ptxas_verbose: bool = False, jobs: int = 4) -> st
         for p in procs:
             if p.wait() != 0:
                 raise RuntimeError("nvcc failed")
-        out = LIB + f".tmp{os.getpid()}"
+        out = target + f".tmp{os.getpid()}"
         subprocess.check_call([cc, *ARCH, "-shared", "-o", out, *objs, "-lcudart_static", "-ldl", "-lpthread",
                                "-lrt"])
-        os.replace(out, LIB)
-    return LIB
+        os.replace(out, target)
+    return target
 
 
 if __name__ == "__main__":

@@ -1,0 +1,339 @@
+// The two passes of the block-energy calibration (explainer §三, offline
+// calibration steps 1-2) on the tensor core: S = Q K^T tile by tile over all
+// key blocks, never storing P.
+//   pass 1 (kLse):    per query row, log2 sum_j 2^(scale' S_ij)  -> lse_ws
+//   pass 2 (kEnergy): per tile, sum_ij 2^(scale' S_ij - lse_i) -> E[r][c], then
+//                     the greedy eps selection of the finished row (select.cuh)
+//
+// CTA (320 threads, one per SM): two query-tile slots; warps 0-3 and 4-7 are
+// the slots' row warpgroups (thread = query row = TMEM lane), warp 8 loads Q
+// and K tiles with TMA, warp 9 issues tcgen05.mma. Tensor memory holds two S
+// buffers per slot (4 x 128 columns), so the MMA of the next tile overlaps
+// the reduction of the current one.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "calibatt.h"
+#include "kernels.h"
+#include "ptx.cuh"
+#include "sched.cuh"
+#include "select.cuh"
+#include "softmax.cuh"
+
+#ifndef CALIBATT_SCORE_EMU
+#define CALIBATT_SCORE_EMU 0x00u
+#endif
+
+namespace calibatt {
+namespace {
+
+constexpr int kScoreThreads = 320;
+constexpr int kScoreRing = 4;               // K tiles in flight
+constexpr int kEnergyScratch = 16384;       // per slot: per-warp tile sums, then sort keys
+// Pairs of a row whose 2^x goes to the FMA-pipe polynomial (bit i%8 of the
+// mask selects pair i) instead of MUFU; measured fastest with none.
+constexpr unsigned kScoreEmu = CALIBATT_SCORE_EMU;
+
+struct ScoreBarriers {
+  uint64_t ring_full[kScoreRing];
+  uint64_t ring_empty[kScoreRing];
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
+  uint64_t s_full[2][2];
+  uint64_t s_empty[2][2];
+  uint64_t mma_done;
+  uint32_t first[kScoreRing];  // ring stage starts a unit (wait for its Q)
+  uint32_t last[kScoreRing];   // ring stage ends a unit (release its Q)
+  uint32_t slot[kScoreRing];
+  uint32_t end;                // producer has no more tiles
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int MODE>
+struct ScoreLayout {
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = 2 * kTile;
+  static constexpr int kAuxOff = kRingOff + kScoreRing * kTile;
+  static constexpr int kAuxBytes = (MODE == kEnergy) ? 2 * kEnergyScratch : 0;
+  static constexpr int kBarOff = kAuxOff + kAuxBytes;
+  static constexpr int kBytes = kBarOff + static_cast<int>(sizeof(ScoreBarriers));
+  static constexpr int kDynSmem = kBytes + 1024;  // + alignment slack
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+    score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ KernelParams p) {
+  using L = ScoreLayout<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sbase = smem_u32(smem);
+  ScoreBarriers& bar = *reinterpret_cast<ScoreBarriers*>(smem + L::kBarOff);
+  volatile int* abort_flag = &bar.abort;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = 2 * gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kScoreRing; ++i) {
+      mbar_init(&bar.ring_full[i], 1);
+      mbar_init(&bar.ring_empty[i], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.q_empty[s], 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&bar.s_full[s][b], 1);
+        mbar_init(&bar.s_empty[s][b], 128);
+      }
+    }
+    mbar_init(&bar.mma_done, 1);
+    bar.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) tmem_alloc(&bar.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+
+  if (warp == 8 && lane == 0) {
+    // ---------------------------------------------------------- TMA producer
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    Cursor cur[2];
+    for (int s = 0; s < 2; ++s) {
+      cur[s].round = 0;
+      cursor_seek(p, 2 * blockIdx.x + s, G, cur[s]);
+    }
+    uint32_t stage = 0, phase = 0, n_q[2] = {0, 0};
+    bool ok = true;
+    while (ok && (cur[0].valid || cur[1].valid)) {
+      for (int s = 0; s < 2 && ok; ++s) {
+        Cursor& c = cur[s];
+        if (!c.valid) continue;
+        if (c.j == 0) {
+          if (!(ok = mbar_wait(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status))) break;
+          uint8_t* dst = smem + L::kQOff + s * kTile;
+          mbar_arrive_expect_tx(&bar.q_full[s], kTile);
+          tma_load_3d(dst, &tm_q, &bar.q_full[s], 0, c.u.r * 128, c.u.hq);
+          tma_load_3d(dst + kHalf, &tm_q, &bar.q_full[s], 64, c.u.r * 128, c.u.hq);
+          ++n_q[s];
+        }
+        if (!(ok = mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status))) break;
+        bar.first[stage] = c.j == 0;
+        bar.last[stage] = c.j == c.u.nnz - 1;
+        bar.slot[stage] = s;
+        uint8_t* dst = smem + L::kRingOff + stage * kTile;
+        mbar_arrive_expect_tx(&bar.ring_full[stage], kTile);
+        tma_load_3d(dst, &tm_k, &bar.ring_full[stage], 0, c.j * 128, c.u.hkv);
+        tma_load_3d(dst + kHalf, &tm_k, &bar.ring_full[stage], 64, c.j * 128, c.u.hkv);
+        if (++stage == kScoreRing) {
+          stage = 0;
+          phase ^= 1;
+        }
+        cursor_next(p, 2 * blockIdx.x + s, G, c);
+      }
+    }
+    if (ok && mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status)) {
+      bar.end = 1;
+      bar.slot[stage] = 2;  // end marker
+      mbar_arrive(&bar.ring_full[stage]);
+    }
+    // no copy may still be landing when the CTA leaves
+    for (int i = 0; i < kScoreRing; ++i) {
+      int st = static_cast<int>(stage) - i;
+      uint32_t ph = phase;
+      if (st < 0) {
+        st += kScoreRing;
+        ph ^= 1;
+      }
+      volatile int never = 0;
+      mbar_wait(&bar.ring_full[st], ph, &never, p.status);
+    }
+    for (int s = 0; s < 2; ++s)
+      if (n_q[s] > 0) {
+        volatile int never = 0;
+        mbar_wait(&bar.q_full[s], (n_q[s] - 1) & 1, &never, p.status);
+      }
+  } else if (warp == 9 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    uint32_t stage = 0, phase = 0, n_q[2] = {0, 0}, n_s[2] = {0, 0};
+    const uint64_t qdesc0 = desc_k_base(sbase + L::kQOff);
+    const uint64_t kdesc0 = desc_k_base(sbase + L::kRingOff);
+    while (true) {
+      if (!mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status)) break;
+      const uint32_t s = *reinterpret_cast<volatile uint32_t*>(&bar.slot[stage]);
+      if (s > 1) break;
+      if (*reinterpret_cast<volatile uint32_t*>(&bar.first[stage])) {
+        if (!mbar_wait(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status)) break;
+      }
+      const int buf = n_s[s] & 1;
+      if (!mbar_wait(&bar.s_empty[s][buf], ((n_s[s] >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + (2 * s + buf) * 128;
+      const uint64_t qd = qdesc0 + s * (kTile >> 4), kd = kdesc0 + stage * (kTile >> 4);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) mma_ss(d_tmem, qd + desc_k_step(ks), kd + desc_k_step(ks), kIdescS, ks > 0);
+      mma_commit(&bar.ring_empty[stage]);
+      if (*reinterpret_cast<volatile uint32_t*>(&bar.last[stage])) {
+        mma_commit(&bar.q_empty[s]);
+        ++n_q[s];
+      }
+      mma_commit(&bar.s_full[s][buf]);
+      ++n_s[s];
+      if (++stage == kScoreRing) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    mma_commit(&bar.mma_done);
+    volatile int never = 0;
+    mbar_wait(&bar.mma_done, 0, &never, p.status);
+  } else if (warp < 8) {
+    // ---------------------------------------------------------- row warpgroups
+    // After a failed wait the warps keep walking their units with every wait
+    // and tensor-memory access skipped, so that the warpgroup's named
+    // barriers are still met by all four warps.
+    const int s = warp >> 2;
+    const int wl = warp & 3;
+    const int row = wl * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
+    const int g = 2 * blockIdx.x + s;
+    const bool ragged_k = (p.n_k & 127) != 0;
+    const int valid_last = p.n_k - (p.nbk - 1) * 128;
+    uint32_t n_sfull = 0;
+    bool ok = true;  // warp-uniform
+    float* part = reinterpret_cast<float*>(smem + L::kAuxOff + s * kEnergyScratch);
+
+    for (int round = 0;; ++round) {
+      Unit u;
+      if (!load_unit(p, unit_index(g, G, round), u)) break;
+      if (!u.write) continue;
+      const int qrow = u.r * 128 + row;
+      const bool row_valid = qrow < p.n_q;
+      float lse2 = 0.f;
+      if (MODE == kEnergy && row_valid) lse2 = p.lse_ws[static_cast<int64_t>(u.hq) * p.nbq * 128 + qrow];
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < u.nnz; ++j) {
+        const int buf = n_sfull & 1;
+        float acc = 0.f;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_full[s][buf], (n_sfull >> 1) & 1, abort_flag,
+                                                       p.status));
+        if (ok) {
+          ++n_sfull;
+          tc_fence_after();
+          float sv[128];
+          tmem_ld128_wait(tmem + lane_off + (2 * s + buf) * 128, sv);
+          tc_fence_before();
+          mbar_arrive(&bar.s_empty[s][buf]);
+          const int nvalid = (ragged_k && j == p.nbk - 1) ? valid_last : 128;
+          if (nvalid < 128) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c >= nvalid) sv[c] = -INFINITY;
+          }
+          float ref;  // subtracted before the exponential
+          if (MODE == kLse) {
+            const float mx = row_max128(sv) * p.scale_log2;
+            const float m_new = fmaxf(m_run, mx);
+            if (m_run != -INFINITY) l_run *= ex2_approx(m_run - m_new);
+            m_run = m_new;
+            ref = m_new;
+          } else {
+            ref = lse2;
+          }
+          if (MODE == kLse || row_valid) {
+            const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 nr2 = make_float2(-ref, -ref);
+            float2 a4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f)};
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              float2 e = exp2_pair<5, kScoreEmu>(i, ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), c2, nr2));
+              if (nvalid < 128) {
+                e.x = 2 * i < nvalid ? e.x : 0.f;
+                e.y = 2 * i + 1 < nvalid ? e.y : 0.f;
+              }
+              a4[i & 3] = fadd2(a4[i & 3], e);
+            }
+            const float2 s01 = fadd2(a4[0], a4[1]), s23 = fadd2(a4[2], a4[3]);
+            acc = (s01.x + s01.y) + (s23.x + s23.y);
+          }
+          if (MODE == kLse) l_run += acc;
+        }
+        if (MODE == kEnergy) {
+          // this warp's share of E[r][j]: sum over its 32 rows
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (lane == 0) part[wl * 1024 + j] = acc;
+        }
+      }
+      if (MODE == kLse) {
+        if (ok) p.lse_ws[static_cast<int64_t>(u.hq) * p.nbq * 128 + qrow] = m_run + log2f(l_run);
+      } else {
+        named_bar_sync(1 + s, 128);
+        const int rows = min(128, p.n_q - u.r * 128);
+        const float inv_rows = 1.f / static_cast<float>(rows);
+        const int64_t erow = (static_cast<int64_t>(u.hq) * p.nbq + u.r) * p.nbk;
+        for (int c = row; c < p.nbk; c += 128) {
+          // fixed summation order: the energy is reproducible run to run
+          const float e = (((part[c] + part[1024 + c]) + part[2048 + c]) + part[3072 + c]) * inv_rows;
+          part[c] = e;
+          if (p.energy && ok) p.energy[erow + c] = e;
+        }
+        if (p.fuse_select) {
+          named_bar_sync(1 + s, 128);
+          SelectOut out{p.mask ? p.mask + erow : nullptr, p.kept ? p.kept + (erow / p.nbk) : nullptr,
+                        p.counts ? p.counts + erow : nullptr};
+          if (!ok) out = SelectOut{nullptr, nullptr, nullptr};
+          select_row(part, p.nbk, p.eps_fx, reinterpret_cast<uint8_t*>(part + 1024),
+                     reinterpret_cast<unsigned long long*>(part + 2048), row, 128, 1 + s, out);
+        }
+        named_bar_sync(1 + s, 128);
+      }
+    }
+  }
+
+  // ---------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int MODE>
+int launch_mode(const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams& p, cudaStream_t stream) {
+  using L = ScoreLayout<MODE>;
+  static_assert(L::kDynSmem <= 232448, "shared memory budget");
+  static bool configured = false;  // per process; the attribute is per function
+  if (!configured) {
+    if (cudaFuncSetAttribute(score_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
+        cudaSuccess)
+      return CALIBATT_ERR_CUDA;
+    configured = true;
+  }
+  if (p.n_units <= 0) return CALIBATT_OK;
+  int grid = (p.n_units + 1) / 2;
+  const int sms = sm_count();
+  if (grid > sms) grid = sms;
+  score_kernel<MODE><<<grid, kScoreThreads, L::kDynSmem, stream>>>(mq, mk, p);
+  return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_score(int mode, const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams& p,
+                 cudaStream_t stream) {
+  return mode == kLse ? launch_mode<kLse>(mq, mk, p, stream) : launch_mode<kEnergy>(mq, mk, p, stream);
+}
+
+}  // namespace calibatt
