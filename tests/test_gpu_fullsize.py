@@ -1,0 +1,179 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark times, on sampled outputs the fp64 oracle computes one by one.
+
+* Wan 2.1 14B 720p: 40 heads x N = 75600 (last block 80 rows); 32 block-sparse
+  heads over random Beta(2,3) masks at 62.5 % sparsity, 8 repeated heads with
+  k = 5 anchor rows of 45; sampled query rows of both kinds.
+* Wan 2.1 14B 480p: calibration energies and fused eps(T/2) selection on
+  sampled block-rows of all 40 heads (N = 32760, last block 120 rows).
+* Mochi 1 480p: masks calibrated on the GPU over 16 inputs at eps = 0.84,
+  aggregated at rho = 0.5, then attention of 20 block-sparse + 4 repeated
+  heads (k = 5 of 30 rows) on sampled rows.
+* Calibration sweep at the Wan-720p shape: eps in {0.84, 0.9, 0.95, 0.99} on
+  sampled block-rows; aggregation of 16 inputs against the oracle aggregator.
+
+Inputs come from the seeded generator (synth), drawn on the device; the
+sampled heads are copied to the host for the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from calibrated_block_sparse_b200 import synth
+from gpu_util import attn_tolerance_ok, compare_masks, require_gpu, tie_affected
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _bits(t):
+    return synth.bf16_bits(t)
+
+
+def _energy_ok(E, E_ref):
+    bound = 2e-5 * E_ref + 2e-6 * E_ref.max(-1, keepdims=True)
+    return bool(np.all(np.abs(E - E_ref) <= bound))
+
+
+def _skiplist(binding, masks, dev):
+    counts = torch.from_numpy(masks.astype(np.int16)).to(dev).view(torch.uint16)
+    _, row_ptr, col_idx, _ = binding.aggregate_masks(counts, 1, 0.5)
+    return row_ptr, col_idx
+
+
+def _sample_rows(rng, heads, n, per_head):
+    rows = []
+    for h in heads:
+        r = rng.choice(n, size=per_head, replace=False)
+        r[0], r[1] = n - 1, 0  # the ragged tail and the first row
+        rows.extend(int(h) * n + r)
+    return np.array(rows, np.int64)
+
+
+def test_wan720_attention_sampled_rows(oracle):
+    binding = require_gpu()
+    wl = synth.WORKLOADS["wan720"]
+    dev = torch.device(DEV)
+    q, k, v = synth.qkv(wl, 7, device=dev)
+    masks = synth.random_block_masks(wl)
+    rep = list(wl.repeat_heads)
+    sparse = [h for h in range(wl.heads) if h not in rep]
+    row_ptr, col_idx = _skiplist(binding, masks, dev)
+    work = torch.from_numpy(binding.build_plan(row_ptr.cpu().numpy(), wl.heads, wl.nb,
+                                               np.array([h not in rep for h in range(wl.heads)], np.uint8))).to(dev)
+    o = torch.zeros_like(q)
+    lse = torch.zeros((wl.heads, wl.n), dtype=torch.float32, device=dev)
+    binding.sparse_attn_fwd(q, k, v, row_ptr, col_idx, work, o=o, lse=lse)
+    binding.repeat_attn_fwd(q, k, v, wl.F, wl.H, wl.W, torch.tensor(rep, dtype=torch.int32, device=dev),
+                            wl.k_anchor, o=o, lse=lse)
+    assert binding.get_status() == 0
+    rng = np.random.default_rng(1)
+    for kind, heads in (("sparse", sparse[::8]), ("repeat", rep[::4])):
+        for h in heads:
+            rows = _sample_rows(rng, [0], wl.n, 24)
+            qh, kh, vh = (_bits(t[h:h + 1]) for t in (q, k, v))
+            if kind == "sparse":
+                o_ref, lse_ref = oracle.masked_attention(qh, kh, vh, masks[h:h + 1], rows=rows)
+            else:
+                o_ref, lse_ref = oracle.repeat_attention(qh, kh, vh, wl.F, wl.H, wl.W, wl.k_anchor, rows=rows)
+            og = o[h].float().cpu().numpy().astype(np.float64)[rows]
+            ok, err, bound = attn_tolerance_ok(og, o_ref)
+            assert ok, (kind, h, err, bound)
+            np.testing.assert_allclose(lse[h].cpu().numpy()[rows], lse_ref, atol=2e-3)
+
+
+def test_wan480_energy_and_selection_sampled_blockrows(oracle):
+    binding = require_gpu()
+    wl = synth.WORKLOADS["wan480"]
+    dev = torch.device(DEV)
+    q, k, _ = synth.qkv(wl, 3, with_v=False, device=dev)
+    eps = binding.eps_schedule(0.84, 0.99, 5, 0.5, 1.0)
+    E, mask, kept, _ = binding.block_energy(q, k, eps=eps)
+    assert binding.get_status() == 0
+    E = E.cpu().numpy().astype(np.float64)
+    mask = mask.cpu().numpy()
+    rng = np.random.default_rng(2)
+    for h in rng.choice(wl.heads, size=3, replace=False):
+        brs = np.array([wl.nb - 1, 0] + list(rng.choice(wl.nb, size=4, replace=False)), np.int64)
+        E_ref = oracle.block_energy(_bits(q[h:h + 1]), _bits(k[h:h + 1]), blockrows=brs)
+        assert _energy_ok(E[h][brs], E_ref), h
+        # fused selection == oracle selection of the same fp32 energies
+        m_same, _, cut = oracle.select(E[h][brs], eps, with_cut=True)
+        assert compare_masks(mask[h][brs], m_same, tie_affected(cut, eps, 1e-6))[2] == 0
+        m_ref, _, cut_ref = oracle.select(E_ref, eps, with_cut=True)
+        assert compare_masks(mask[h][brs], m_ref, tie_affected(cut_ref, eps, 1e-4))[2] == 0
+
+
+def test_calib720_eps_sweep_and_aggregation(oracle):
+    binding = require_gpu()
+    wl = synth.WORKLOADS["calib720"]
+    heads = [0, 17]  # a subset of heads at the full sequence length
+    dev = torch.device(DEV)
+    rng = np.random.default_rng(3)
+    brs = np.array([wl.nb - 1, 0] + list(rng.choice(wl.nb, size=2, replace=False)), np.int64)
+    n_in, rho = 16, 0.5
+    counts = torch.zeros((len(heads), wl.nb, wl.nb), dtype=torch.uint16, device=dev)
+    per_input = []
+    for p in range(n_in):
+        q, k, _ = synth.qkv(wl, p, heads=heads, with_v=False, device=dev)
+        if p == 0:
+            E, _, _, _ = binding.block_energy(q, k)
+            E = E.cpu().numpy().astype(np.float64)
+            E_ref = oracle.block_energy(_bits(q[:1]), _bits(k[:1]), blockrows=brs)
+            assert _energy_ok(E[0][brs], E_ref)
+            for eps in (0.84, 0.9, 0.95, 0.99):
+                _, m, _, _ = binding.block_energy(q, k, eps=eps, energy=False)
+                m = m.cpu().numpy()[0][brs]
+                m_same, _, cut = oracle.select(E[0][brs], eps, with_cut=True)
+                assert compare_masks(m, m_same, tie_affected(cut, eps, 1e-6))[2] == 0
+                m_ref, _, cut_ref = oracle.select(E_ref, eps, with_cut=True)
+                assert compare_masks(m, m_ref, tie_affected(cut_ref, eps, 1e-4))[2] == 0
+        m_p = torch.zeros((len(heads), wl.nb, wl.nb), dtype=torch.uint8, device=dev)
+        binding.block_energy(q, k, eps=0.9, energy=False, mask=m_p, counts=counts)
+        per_input.append(m_p.cpu().numpy())
+    assert binding.get_status() == 0
+    mask, row_ptr, col_idx, nnz = binding.aggregate_masks(counts, n_in, rho)
+    m_ref, c_ref = oracle.aggregate(np.stack(per_input), rho)
+    np.testing.assert_array_equal(counts.cpu().numpy().astype(np.int32), c_ref)
+    np.testing.assert_array_equal(mask.cpu().numpy(), m_ref)
+    rp_ref, ci_ref = oracle.mask_to_csr(m_ref)
+    np.testing.assert_array_equal(row_ptr.cpu().numpy(), rp_ref)
+    np.testing.assert_array_equal(col_idx.cpu().numpy(), ci_ref)
+
+
+def test_mochi_calibrated_attention_sampled_rows(oracle):
+    binding = require_gpu()
+    wl = synth.WORKLOADS["mochi480"]
+    dev = torch.device(DEV)
+    n_in, eps, rho = 16, 0.84, 0.5
+    counts = torch.zeros((wl.heads, wl.nb, wl.nb), dtype=torch.uint16, device=dev)
+    for p in range(n_in):
+        q, k, _ = synth.qkv(wl, p, with_v=False, device=dev)
+        binding.block_energy(q, k, eps=eps, energy=False, counts=counts)
+    mask, row_ptr, col_idx, _ = binding.aggregate_masks(counts, n_in, rho)
+    assert binding.get_status() == 0
+    m = mask.cpu().numpy()
+    rep = list(wl.repeat_heads)
+    sparse = [h for h in range(wl.heads) if h not in rep]
+    sparsity = 1.0 - float(np.mean([m[h].mean() for h in sparse]))
+    print(f"mochi calibrated sparsity {sparsity:.3f}")
+    work = torch.from_numpy(binding.build_plan(row_ptr.cpu().numpy(), wl.heads, wl.nb,
+                                               np.array([h not in rep for h in range(wl.heads)], np.uint8))).to(dev)
+    q, k, v = synth.qkv(wl, n_in, device=dev)
+    o = torch.zeros_like(q)
+    binding.sparse_attn_fwd(q, k, v, row_ptr, col_idx, work, o=o)
+    binding.repeat_attn_fwd(q, k, v, wl.F, wl.H, wl.W, torch.tensor(rep, dtype=torch.int32, device=dev),
+                            wl.k_anchor, o=o)
+    assert binding.get_status() == 0
+    rng = np.random.default_rng(4)
+    for h in (sparse[0], sparse[11], rep[0], rep[-1]):
+        rows = _sample_rows(rng, [0], wl.n, 24)
+        qh, kh, vh = (_bits(t[h:h + 1]) for t in (q, k, v))
+        if h in rep:
+            o_ref, _ = oracle.repeat_attention(qh, kh, vh, wl.F, wl.H, wl.W, wl.k_anchor, rows=rows)
+        else:
+            o_ref, _ = oracle.masked_attention(qh, kh, vh, m[h:h + 1], rows=rows)
+        og = o[h].float().cpu().numpy().astype(np.float64)[rows]
+        ok, err, bound = attn_tolerance_ok(og, o_ref)
+        assert ok, (h, err, bound)
