@@ -165,3 +165,23 @@ def test_tiny_calibration_pipeline(oracle):
     o_ref, _ = oracle.masked_attention(synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v),
                                        mask.cpu().numpy())
     assert attn_tolerance_ok(bf16_to_f64(o), o_ref)[0]
+
+
+def test_calibrate_sharded_single_rank_matches_oracle(oracle):
+    """The multi-GPU calibration entry on one rank (no process group)."""
+    binding = require_gpu()
+    from calibrated_block_sparse_b200 import multi
+    wl = synth.WORKLOADS["tiny"]
+    dev = torch.device("cuda")
+    inputs = {p: synth.qkv(wl, p, with_v=False) for p in range(4)}
+    mask, row_ptr, col_idx, _ = multi.calibrate_sharded(
+        lambda p: (inputs[p][0].to(dev), inputs[p][1].to(dev)), wl.heads, wl.nb, 4, 0.9, 0.5, device=dev)
+    ref = []
+    ties = 0
+    for p in range(4):
+        E_ref = oracle.block_energy(synth.bf16_bits(inputs[p][0]), synth.bf16_bits(inputs[p][1]))
+        m, _, cut = oracle.select(E_ref, 0.9, with_cut=True)
+        ref.append(m)
+        ties += int(tie_affected(cut, 0.9, 1e-4).sum())
+    m_ref, _ = oracle.aggregate(np.stack(ref), 0.5)
+    assert int(np.sum(mask.cpu().numpy() != m_ref)) <= ties
