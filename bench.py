@@ -249,16 +249,24 @@ def run_ours(args, world, rank, local):
     sparse_heads = [h for h in range(heads) if h not in rep_heads]
 
     # inputs: resident in HBM before the timed region
-    q, k, v = synth.qkv(wl, 1000 + rank, device=dev)
     if args.workload == "wan720":
+        # random per-head masks at 62.5 % sparsity; skip lists built on the GPU
+        # by the aggregation kernel (one input, rho 0.5)
         masks = synth.random_block_masks(synth.WORKLOADS["wan720"])[:heads]
+        counts = torch.from_numpy(masks.astype(np.int16)).to(dev).view(torch.uint16)
+        mask_d, row_ptr, col_idx, _ = binding.aggregate_masks(counts, 1, 0.5)
     else:
-        masks = (np.random.default_rng(7).random((heads, nb, nb)) < 0.32).astype(np.uint8)
-        masks[:, np.arange(nb), np.arange(nb)] = 1
-    # skip lists built on the GPU by the aggregation kernel (one input, rho 0.5)
-    counts = torch.from_numpy(masks.astype(np.int16)).to(dev).view(torch.uint16)
-    mask_d, row_ptr, col_idx, _ = binding.aggregate_masks(counts, 1, 0.5)
-    binding.check_status(what="aggregate_masks")
+        # masks calibrated on the GPU over the workload's seeded inputs
+        n_cal, eps_cal = synth.CALIBRATION[args.workload]
+        counts = torch.zeros((heads, nb, nb), dtype=torch.uint16, device=dev)
+        for pi in range(n_cal):
+            qc, kc, _ = synth.qkv(wl, pi, with_v=False, device=dev)
+            binding.block_energy(qc, kc, eps=eps_cal, energy=False, counts=counts)
+            del qc, kc
+        mask_d, row_ptr, col_idx, _ = binding.aggregate_masks(counts, n_cal, 0.5)
+        masks = mask_d.cpu().numpy()
+    binding.check_status(what="skip lists")
+    q, k, v = synth.qkv(wl, 1000 + rank, device=dev)
     row_ptr_h = row_ptr.cpu().numpy()
     head_active = np.array([h not in rep_heads for h in range(heads)], np.uint8)
     work = torch.from_numpy(binding.build_plan(row_ptr_h, heads, nb, head_active)).to(dev)
