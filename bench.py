@@ -234,6 +234,29 @@ def cuda_time(fn, reps, stream):
     return start.elapsed_time(end) / reps
 
 
+def graph_time(fn, reps, stream):
+    """Average device ms of fn() for kernels too short to time one by one: the
+    reps calls are captured in a CUDA graph and replayed, so host launch
+    overhead does not open gaps between them."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    g.replay()
+    end.record(stream)
+    end.synchronize()
+    ms = start.elapsed_time(end) / reps
+    del g
+    return ms
+
+
 def run_ours(args, world, rank, local):
     from calibrated_block_sparse_b200 import binding
     binding.load()
@@ -382,11 +405,13 @@ def run_ours(args, world, rank, local):
         f_energy_alg = float(2 * D * n * n * ch)  # one S = Q K^T per input
         f_energy_issued = 2 * f_energy_alg        # two passes recompute S
 
-        def select_call():
-            binding.select_mask(energy, 0.9, mask=cmask, kept=False, stream=stream)
+        gstream = torch.cuda.Stream()
 
-        select_call()
-        s_ms = cuda_time(select_call, 5, stream)
+        def select_call():
+            binding.select_mask(energy, 0.9, mask=cmask, kept=False, stream=torch.cuda.current_stream())
+
+        with torch.cuda.stream(gstream):
+            s_ms = graph_time(select_call, 20, gstream)
         sel_bytes = ch * nb * nb * (4 + 1)
         agg_ws = torch.empty(binding.load().calibatt_aggregate_workspace_size(ch, nb), dtype=torch.uint8, device=dev)
         am = torch.empty((ch, nb, nb), dtype=torch.uint8, device=dev)
@@ -398,10 +423,11 @@ def run_ours(args, world, rank, local):
         def agg_call():
             lib.calibatt_aggregate_masks(binding._ptr(ccounts), 64, ch, nb, 0.5, binding._ptr(am),
                                          binding._ptr(arp), binding._ptr(aci), aci.numel(), binding._ptr(annz),
-                                         binding._ptr(agg_ws), agg_ws.numel(), binding._stream(stream))
+                                         binding._ptr(agg_ws), agg_ws.numel(),
+                                         binding._stream(torch.cuda.current_stream()))
 
-        agg_call()
-        a_ms = cuda_time(agg_call, 5, stream)
+        with torch.cuda.stream(gstream):
+            a_ms = graph_time(agg_call, 20, gstream)
         binding.check_status(what="calibration")
         kept_agg = int(annz.item())
         agg_bytes = ch * nb * nb * (2 + 1 + 1) + kept_agg * 4 + (ch * nb + 1) * 4 * 3

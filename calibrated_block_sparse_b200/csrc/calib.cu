@@ -14,18 +14,21 @@ namespace calibatt {
 
 
 // ------------------------------------------------------------------ selection
-// One 128-thread CTA per block-row of energies.
-__global__ void __launch_bounds__(128) select_kernel(const float* __restrict__ energy, int nb, long long eps_fx,
-                                                     uint8_t* mask, int32_t* kept, uint16_t* counts) {
-  __shared__ float e_row[1024];
-  __shared__ __align__(16) uint8_t aux[4096];
-  __shared__ unsigned long long keys[1024];
-  const int64_t row = blockIdx.x;
+// One warp per block-row of energies, four rows per CTA; no block barriers.
+// PER (columns per lane, >= nb / 32) sizes the per-lane register arrays.
+template <int PER>
+__global__ void __launch_bounds__(128) select_kernel(const float* __restrict__ energy, int64_t rows, int nb,
+                                                     long long eps_fx, uint8_t* mask, int32_t* kept,
+                                                     uint16_t* counts) {
+  __shared__ float e_rows[4][1024];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + w;
+  if (row >= rows) return;
   const float* src = energy + row * nb;
-  for (int c = threadIdx.x; c < nb; c += 128) e_row[c] = src[c];
-  __syncthreads();
+  for (int c = lane; c < nb; c += 32) e_rows[w][c] = src[c];
+  __syncwarp();
   SelectOut out{mask ? mask + row * nb : nullptr, kept ? kept + row : nullptr, counts ? counts + row * nb : nullptr};
-  select_row(e_row, nb, eps_fx, aux, keys, threadIdx.x, 128, 1, out);
+  select_row<PER>(e_rows[w], nb, eps_fx, nullptr, lane, 32, 0, out);
 }
 
 // ------------------------------------------------------------------ accumulation
@@ -149,7 +152,15 @@ namespace calibatt {
 int launch_select(const float* energy, int64_t rows, int nb, long long eps_fx, uint8_t* mask, int32_t* kept,
                   uint16_t* counts, cudaStream_t stream) {
   if (rows <= 0) return CALIBATT_OK;
-  select_kernel<<<static_cast<unsigned>(rows), 128, 0, stream>>>(energy, nb, eps_fx, mask, kept, counts);
+  const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
+  if (nb <= 256)
+    select_kernel<8><<<grid, 128, 0, stream>>>(energy, rows, nb, eps_fx, mask, kept, counts);
+  else if (nb <= 512)
+    select_kernel<16><<<grid, 128, 0, stream>>>(energy, rows, nb, eps_fx, mask, kept, counts);
+  else if (nb <= 768)
+    select_kernel<24><<<grid, 128, 0, stream>>>(energy, rows, nb, eps_fx, mask, kept, counts);
+  else
+    select_kernel<32><<<grid, 128, 0, stream>>>(energy, rows, nb, eps_fx, mask, kept, counts);
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
 }
 

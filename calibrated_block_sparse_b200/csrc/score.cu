@@ -32,7 +32,7 @@ namespace {
 
 constexpr int kScoreThreads = 320;
 constexpr int kScoreRing = 4;               // K tiles in flight
-constexpr int kEnergyScratch = 16384;       // per slot: per-warp tile sums, then sort keys
+constexpr int kEnergyScratch = 16384;       // per slot: per-warp tile sums, then selection scratch
 // Pairs of a row whose 2^x goes to the FMA-pipe polynomial (bit i%8 of the
 // mask selects pair i) instead of MUFU; measured fastest with none.
 constexpr unsigned kScoreEmu = CALIBATT_SCORE_EMU;
@@ -292,8 +292,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           SelectOut out{p.mask ? p.mask + erow : nullptr, p.kept ? p.kept + (erow / p.nbk) : nullptr,
                         p.counts ? p.counts + erow : nullptr};
           if (!ok) out = SelectOut{nullptr, nullptr, nullptr};
-          select_row(part, p.nbk, p.eps_fx, reinterpret_cast<uint8_t*>(part + 1024),
-                     reinterpret_cast<unsigned long long*>(part + 2048), row, 128, 1 + s, out);
+          select_row<8>(part, p.nbk, p.eps_fx, reinterpret_cast<uint8_t*>(part + 1024), row, 128, 1 + s, out);
         }
         named_bar_sync(1 + s, 128);
       }

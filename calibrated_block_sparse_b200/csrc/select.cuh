@@ -1,12 +1,18 @@
 // Greedy eps selection of one block-row, run cooperatively by T threads of a
 // CTA (explainer §三, step 3: keep the fewest key blocks whose cumulative
-// energy reaches eps).
+// energy reaches eps; greedy order: energy descending, equal energies by lower
+// column first).
 //
-// Order: energy descending, equal energies by lower column (a 64-bit key
-// (~bits(E), col) sorted ascending by a bitonic network in shared memory).
-// Running sums are exact: every energy is converted to an integer with 50
-// fraction bits (truncated), so the parallel prefix scan gives the same cut as
-// a sequential sum in the same order.
+// No sort is needed. With every energy taken exactly in fixed point (50
+// fraction bits, truncated), the greedy cut is determined by the energy tau
+// of the block at which the running sum first reaches eps:
+//   tau = the largest energy v with  S(v) = sum_{E >= v} fx(E) >= eps_fx.
+// S is non-increasing in v and the float bit patterns of non-negative
+// energies order like their values, so tau is found by a binary search over
+// bit patterns, each step one exact integer sum over the row. The kept set is
+// every block with E > tau plus the first r blocks (in column order) with
+// E == tau, r the fewest that reach eps. Because the sums are exact integers,
+// the result equals a sequential greedy sum in sorted order.
 #pragma once
 #include <cstdint>
 
@@ -39,100 +45,180 @@ __device__ __forceinline__ long long energy_fixed(float e) {
   return static_cast<long long>(man >> (-sh));
 }
 
-__device__ __forceinline__ unsigned long long energy_key(float e, int col) {
-  return (static_cast<unsigned long long>(0xFFFFFFFFu - __float_as_uint(e)) << 32) | static_cast<uint32_t>(col);
-}
-
 __device__ __forceinline__ void group_sync(int bar_id, int T) {
-  asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(T) : "memory");
+  if (T == 32)
+    __syncwarp();
+  else
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(T) : "memory");
 }
 
-// E: shared [nb] energies; aux: shared scratch >= 4 KB; keys: shared [1024].
-// Every one of the T threads (T a multiple of 32, <= 1024) must call this.
-static __device__ __noinline__ void select_row(const float* E, int nb, long long eps_fx, uint8_t* aux,
-                                        unsigned long long* keys, int tid, int T, int bar_id, SelectOut out) {
-  uint8_t* keep = aux;                                              // [1024]
-  long long* warp_tot = reinterpret_cast<long long*>(aux + 1024);  // [32]
-  int* first_hit = reinterpret_cast<int*>(aux + 1024 + 256);
-  int* nonzero = first_hit + 1;
+// Per-warp partials for reductions over T > 32 threads.
+struct SelectScratch {
+  long long wsum[32];
+  int wcnt[32];
+};
 
-  int npow = 2;
-  while (npow < nb) npow <<= 1;
-  for (int i = tid; i < npow; i += T) keys[i] = (i < nb) ? energy_key(clamp_energy(E[i]), i) : ~0ull;
-  for (int i = tid; i < nb; i += T) keep[i] = 0;
-  if (tid == 0) {
-    *first_hit = 0x7FFFFFFF;
-    *nonzero = 0;
+// Sum of a per-thread int64 and int over the T threads (T multiple of 32).
+__device__ __forceinline__ void group_sum(long long& v, int& c, SelectScratch* sc, int tid, int T, int bar_id) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v += __shfl_xor_sync(0xffffffffu, v, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  if (T == 32) return;
+  if ((tid & 31) == 0) {
+    sc->wsum[tid >> 5] = v;
+    sc->wcnt[tid >> 5] = c;
   }
   group_sync(bar_id, T);
+  v = 0;
+  c = 0;
+  for (int w = 0; w < (T >> 5); ++w) {
+    v += sc->wsum[w];
+    c += sc->wcnt[w];
+  }
+  group_sync(bar_id, T);
+}
 
-  // bitonic sort, ascending keys
-  for (int k = 2; k <= npow; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < npow; i += T) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long a = keys[i], b = keys[ixj];
-          const bool up = (i & k) == 0;
-          if ((a > b) == up) {
-            keys[i] = b;
-            keys[ixj] = a;
-          }
-        }
-      }
-      group_sync(bar_id, T);
+// Max of a per-thread key over the T threads.
+__device__ __forceinline__ unsigned long long group_max(unsigned long long v, SelectScratch* sc, int tid, int T,
+                                                        int bar_id) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long u = __shfl_xor_sync(0xffffffffu, v, o);
+    v = u > v ? u : v;
+  }
+  if (T == 32) return v;
+  if ((tid & 31) == 0) sc->wsum[tid >> 5] = static_cast<long long>(v);
+  group_sync(bar_id, T);
+  v = 0;
+  for (int w = 0; w < (T >> 5); ++w) {
+    const unsigned long long u = static_cast<unsigned long long>(sc->wsum[w]);
+    v = u > v ? u : v;
+  }
+  group_sync(bar_id, T);
+  return v;
+}
+
+// E: shared [nb] energies; aux: shared scratch of sizeof(SelectScratch)
+// (unused when T == 32). Every one of the T threads (T a multiple of 32,
+// nb <= PER * T) must call this. Thread tid owns columns tid*per .. +per-1.
+template <int PER>
+__device__ __forceinline__ void select_row(const float* E, int nb, long long eps_fx, uint8_t* aux, int tid, int T,
+                                           int bar_id, SelectOut out) {
+  SelectScratch* sc = reinterpret_cast<SelectScratch*>(aux);
+  const int per = (nb + T - 1) / T;
+  const int c0 = tid * per;
+  uint32_t bits[PER];
+  long long fx[PER];
+  long long tot = 0;
+  int nz = 0;
+  // top block key (bits, inverted column): the largest energy, lowest column
+  unsigned long long top = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int c = c0 + i;
+    const bool in = i < per && c < nb;
+    const float e = in ? clamp_energy(E[c]) : 0.f;
+    bits[i] = __float_as_uint(e);
+    fx[i] = energy_fixed(e);
+    tot += fx[i];
+    nz += e > 0.f;
+    if (in) {
+      const unsigned long long key = (static_cast<unsigned long long>(bits[i]) << 32) | (0xFFFFFFFFu - c);
+      top = key > top ? key : top;
     }
   }
+  top = group_max(top, sc, tid, T, bar_id);
+  group_sum(tot, nz, sc, tid, T, bar_id);
+  const int top_col = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(top));
+  const uint32_t top_bits = static_cast<uint32_t>(top >> 32);
 
-  // exact prefix sums of the sorted energies: contiguous chunk per thread
-  const int per = (nb + T - 1) / T;
-  const int i0 = tid * per;
-  const int i1 = min(nb, i0 + per);
-  long long local = 0;
-  int nz = 0;
-  for (int i = i0; i < i1; ++i) {
-    const float e = __uint_as_float(0xFFFFFFFFu - static_cast<uint32_t>(keys[i] >> 32));
-    local += energy_fixed(e);
-    nz += e > 0.f;
+  // 0 = the single top block, 1 = every nonzero block, 2 = greedy cut at tau
+  int mode = 2;
+  if (eps_fx <= 0 || nz == 0) mode = 0;
+  else if (tot < eps_fx) mode = 1;
+
+  uint32_t tau = 0;
+  long long above = 0;  // sum of fx over blocks with energy > tau
+  if (mode == 2) {
+    // largest b in [0, top_bits] with S(b) >= eps (S(0) = tot >= eps)
+    uint32_t lo = 0, hi = top_bits;
+    while (lo < hi) {
+      const uint32_t mid = lo + (hi - lo + 1) / 2;
+      long long sm = 0;
+      int dummy = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) sm += bits[i] >= mid ? fx[i] : 0;
+      group_sum(sm, dummy, sc, tid, T, bar_id);
+      if (sm >= eps_fx)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    tau = lo;
+    int dummy = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) above += bits[i] > tau ? fx[i] : 0;
+    group_sum(above, dummy, sc, tid, T, bar_id);
   }
-  // exclusive scan of the per-thread totals: shuffles inside a warp, then warps
+
+  // rank of each block among the blocks equal to tau, in column order
+  int n_eq = 0;
+  if (mode == 2) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) n_eq += (i < per && c0 + i < nb && bits[i] == tau);
+  }
   const int lane = tid & 31, w = tid >> 5;
-  long long incl = local;
+  int incl = n_eq;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  if (lane == 31) warp_tot[w] = incl;
-  if (nz) atomicAdd(nonzero, nz);
-  group_sync(bar_id, T);
-  long long run = incl - local;
-  for (int ww = 0; ww < w; ++ww) run += warp_tot[ww];
-  for (int i = i0; i < i1; ++i) {
-    const float e = __uint_as_float(0xFFFFFFFFu - static_cast<uint32_t>(keys[i] >> 32));
-    run += energy_fixed(e);
-    if (run >= eps_fx) {
-      atomicMin(first_hit, i + 1);
-      break;
-    }
+  int rank = incl - n_eq;
+  if (T > 32) {
+    if (lane == 31) sc->wcnt[w] = incl;
+    group_sync(bar_id, T);
+    for (int ww = 0; ww < w; ++ww) rank += sc->wcnt[ww];
+    group_sync(bar_id, T);  // every rank read before the partials are reused
   }
-  group_sync(bar_id, T);
-  int m = *first_hit;
-  if (m == 0x7FFFFFFF) m = *nonzero;  // eps not reached: every nonzero-energy block
-  if (m < 1) m = 1;
-  if (m > nb) m = nb;
-  for (int i = tid; i < m; i += T) keep[static_cast<uint32_t>(keys[i])] = 1;
-  group_sync(bar_id, T);
-  for (int c = tid; c < nb; c += T) {
-    const uint8_t kbit = keep[c];
-    if (out.mask) out.mask[c] = kbit;
-    if (out.counts && kbit) {
+  long long r_need = 0;
+  if (mode == 2) {
+    const long long ft = energy_fixed(__uint_as_float(tau));
+    r_need = ft > 0 ? (eps_fx - above + ft - 1) / ft : 1;
+  }
+  int kept_mine = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int c = c0 + i;
+    if (i >= per || c >= nb) continue;
+    bool k;
+    if (mode == 0) {
+      k = (c == top_col);
+    } else if (mode == 1) {
+      k = bits[i] > 0;
+    } else if (bits[i] > tau) {
+      k = true;
+    } else if (bits[i] == tau) {
+      k = rank < r_need;
+      ++rank;
+    } else {
+      k = false;
+    }
+    kept_mine += k;
+    if (out.mask) out.mask[c] = k ? 1 : 0;
+    if (out.counts && k) {
       const uint16_t old = out.counts[c];
       if (old != 0xFFFFu) out.counts[c] = old + 1;
     }
   }
-  if (tid == 0 && out.kept) *out.kept = m;
-  group_sync(bar_id, T);
+  if (out.kept) {
+    long long dummy = 0;
+    group_sum(dummy, kept_mine, sc, tid, T, bar_id);
+    if (tid == 0) *out.kept = kept_mine;
+  }
+  (void)top_bits;
 }
 
 }  // namespace calibatt

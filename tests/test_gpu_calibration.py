@@ -185,3 +185,21 @@ def test_calibrate_sharded_single_rank_matches_oracle(oracle):
         ties += int(tie_affected(cut, 0.9, 1e-4).sum())
     m_ref, _ = oracle.aggregate(np.stack(ref), 0.5)
     assert int(np.sum(mask.cpu().numpy() != m_ref)) <= ties
+
+
+@pytest.mark.parametrize("nb", [7, 64, 591, 1024])
+def test_select_with_many_equal_energies_is_exact(oracle, nb):
+    """Energies from a coarse grid (multiples of 1/64) make long runs of equal
+    values at the cut; eps sits between grid points, so no row is tie-affected
+    and the GPU's cut (largest tau, then lowest columns) must equal the
+    oracle's stable greedy order exactly."""
+    binding = require_gpu()
+    rng = np.random.default_rng(nb)
+    heads = 2
+    E = (rng.integers(0, 5, size=(heads, nb, nb)) / 64.0).astype(np.float32)
+    dev = torch.device("cuda")
+    for eps in (0.3 + 1 / 128, 0.7 + 1 / 128, 2.0 + 1 / 256):
+        mask, kept, _ = binding.select_mask(torch.from_numpy(E).to(dev), eps)
+        m_ref, kept_ref = oracle.select(E.astype(np.float64), eps)
+        np.testing.assert_array_equal(mask.cpu().numpy(), m_ref)
+        np.testing.assert_array_equal(kept.cpu().numpy(), kept_ref)
