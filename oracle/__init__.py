@@ -69,6 +69,10 @@ def _load():
             lib.oracle_mask_to_csr.restype = i64
             lib.oracle_eps_schedule.argtypes = [f64, f64, f64, f64, f64]
             lib.oracle_eps_schedule.restype = f64
+            lib.oracle_pixel_row_energy.argtypes = [P, P, i32, i32, i32, i32, i32, i32, f64, P, i64, P, i32]
+            lib.oracle_pixel_row_energy.restype = None
+            lib.oracle_spatial_score.argtypes = [P, i32, i32, i64, i32]
+            lib.oracle_spatial_score.restype = f64
             _lib = lib
     return _lib
 
@@ -239,3 +243,42 @@ def mask_to_csr(mask):
 def eps_schedule(A, C, k, t, T):
     """eps(t) = A + (C - A) exp(-k t / T) (explainer §三)."""
     return _load().oracle_eps_schedule(float(A), float(C), float(k), float(t), float(T))
+
+
+def pixel_row_energy(q, k, F, H, W, B=128, scale=None, prows=None, threads=None):
+    """Block-energy profile of every pixel row R = (f, r) of a frame:
+    Epx[R][c] = (1/W) sum over the W queries of R and the keys of block c of
+    softmax(scale QK^T) (the block energy of explainer §三 step 2, taken over
+    pixel rows instead of query blocks; §二 observation 4).
+
+    ``prows``: optional int64 array of h*F*H + R; default all (returns [h][F*H][nb])."""
+    q, k = _bf16_bits(q), _bf16_bits(k)
+    h, n, d = q.shape
+    assert n == F * H * W
+    nb = (n + B - 1) // B
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    if prows is None:
+        pr, npr = None, h * F * H
+    else:
+        pr = np.ascontiguousarray(prows, dtype=np.int64)
+        npr = pr.size
+    E = np.empty((npr, nb), np.float64)
+    _load().oracle_pixel_row_energy(_ptr(q), _ptr(k), h, F, H, W, d, B, scale, _ptr(pr), npr, _ptr(E),
+                                    _threads(threads))
+    return E.reshape(h, F * H, nb) if prows is None else E
+
+
+def spatial_score(Epx, F, H, k_anchor=5):
+    """s of one head: mean over frames and non-anchor rows of the cosine
+    similarity between a pixel row's profile and its nearest anchor row's
+    (explainer §三, the spatial similarity score; the pages give no formula)."""
+    E = np.ascontiguousarray(Epx, dtype=np.float64)
+    assert E.ndim == 2 and E.shape[0] == F * H
+    if not 1 <= k_anchor <= H:
+        raise ValueError("k_anchor must be in [1, H]")
+    return _load().oracle_spatial_score(_ptr(E), F, H, E.shape[1], k_anchor)
+
+
+def repeat_flag(s, gamma=0.87):
+    """A head is spatially repeated when its score exceeds gamma (explainer §三)."""
+    return bool(s > gamma)

@@ -386,3 +386,90 @@ int64_t oracle_mask_to_csr(const uint8_t *mask, int heads, int64_t nb, int32_t *
 double oracle_eps_schedule(double A, double C, double k, double t, double T) {
     return A + (C - A) * exp(-k * t / T);
 }
+
+/* ------------------------------------------------------------------------ */
+/* 7. Spatial similarity score of a head (explainer §三: a score s^(t,l,h)   */
+/*    per head, flagged as spatially repeated when it exceeds gamma = 0.87;  */
+/*    §二 observation 4 and §六: the pixel rows of a frame attend alike, so  */
+/*    the k anchor rows can stand in for the rest).  The pages give no      */
+/*    formula for s.  Reading used here:                                     */
+/*      pixel row R = (f, r) holds the W queries i = f*H*W + r*W + c;         */
+/*      its block-energy profile over the key blocks J_c' is                 */
+/*        Epx[R][c'] = (1/W) sum_{i in R} sum_{j in J_c'} P_ij,              */
+/*      P = softmax(scale Q K^T) over all n keys (as for the block energy);   */
+/*      s = mean over frames f and non-anchor rows r of                      */
+/*          cos(Epx[(f, r)], Epx[(f, a(r))]),  a(r) the row's nearest anchor  */
+/*          (the row whose output the repeated head copies to it).           */
+/*    A head whose every row is an anchor (k = H) has s = 1; a cosine with a */
+/*    zero profile counts as 0.                                              */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    const uint16_t *q, *k;
+    int d, B, W;
+    int64_t n, nb, n_prow; /* pixel rows per head = F*H */
+    double scale;
+    const int64_t *prows;
+    double *Epx;
+} prow_ctx;
+
+static void prow_energy_row(void *vctx, int64_t idx, double *s) {
+    prow_ctx *c = (prow_ctx *)vctx;
+    int64_t g = c->prows ? c->prows[idx] : idx; /* h * n_prow + R */
+    int64_t h = g / c->n_prow, R = g % c->n_prow;
+    double *Er = c->Epx + idx * c->nb;
+    for (int64_t cc = 0; cc < c->nb; ++cc) Er[cc] = 0.0;
+    for (int64_t i = R * c->W; i < (R + 1) * c->W; ++i) {
+        const uint16_t *qi = c->q + (h * c->n + i) * c->d;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < c->n; ++j) {
+            const uint16_t *kj = c->k + (h * c->n + j) * c->d;
+            double dot = 0.0;
+            for (int u = 0; u < c->d; ++u) dot += bf16_to_double(qi[u]) * bf16_to_double(kj[u]);
+            s[j] = c->scale * dot;
+            if (s[j] > m) m = s[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < c->n; ++j) l += exp(s[j] - m);
+        double lse_i = m + log(l);
+        for (int64_t j = 0; j < c->n; ++j) Er[j / c->B] += exp(s[j] - lse_i);
+    }
+    for (int64_t cc = 0; cc < c->nb; ++cc) Er[cc] /= (double)c->W;
+}
+
+void oracle_pixel_row_energy(const uint16_t *q, const uint16_t *k, int heads, int F, int H, int W, int d,
+                             int B, double scale, const int64_t *prows, int64_t n_prows, double *Epx,
+                             int threads) {
+    int64_t n = (int64_t)F * H * W;
+    prow_ctx c = {q, k, d, B, W, n, (n + B - 1) / B, (int64_t)F * H, scale, prows, Epx};
+    if (!prows) n_prows = (int64_t)heads * F * H;
+    run_rows(prow_energy_row, &c, n_prows, threads, (size_t)n);
+}
+
+/* s of one head from its profiles Epx [F*H][nb]. */
+double oracle_spatial_score(const double *Epx, int F, int H, int64_t nb, int k_anchor) {
+    int *anchors = (int *)malloc(sizeof(int) * (size_t)k_anchor);
+    int *owner = (int *)malloc(sizeof(int) * (size_t)H);
+    oracle_anchor_rows(H, k_anchor, anchors);
+    oracle_nearest_anchor(H, k_anchor, anchors, owner);
+    double total = 0.0;
+    int64_t count = 0;
+    for (int f = 0; f < F; ++f) {
+        for (int r = 0; r < H; ++r) {
+            int a = anchors[owner[r]];
+            if (a == r) continue; /* an anchor row is computed, not copied */
+            const double *x = Epx + ((int64_t)f * H + r) * nb;
+            const double *y = Epx + ((int64_t)f * H + a) * nb;
+            double xy = 0.0, xx = 0.0, yy = 0.0;
+            for (int64_t c = 0; c < nb; ++c) {
+                xy += x[c] * y[c];
+                xx += x[c] * x[c];
+                yy += y[c] * y[c];
+            }
+            total += (xx > 0.0 && yy > 0.0) ? xy / (sqrt(xx) * sqrt(yy)) : 0.0;
+            ++count;
+        }
+    }
+    free(anchors);
+    free(owner);
+    return count ? total / (double)count : 1.0;
+}
