@@ -68,6 +68,8 @@ def load(build_if_missing: bool = False):
             "calibatt_aggregate_workspace_size": (sz, [i32, i32]),
             "calibatt_aggregate_masks": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P, sz, P]),
             "calibatt_aggregate_masks_noalloc": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P]),
+            "calibatt_pixel_row_energy": (i32, [P, P, i32, i32, i32, i32, i32, f32, P, P, P, P]),
+            "calibatt_spatial_score": (i32, [P, i32, i32, i32, i32, i32, f32, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -231,6 +233,49 @@ def block_energy(q, k, eps=None, energy=True, mask=None, kept=None, counts=None,
                                       _ptr(counts), _stream(stream))
     _check(rc, "calibatt_block_energy")
     return e, mask, kept, counts
+
+
+def pixel_row_energy(q, k, F, H, W, energy=False, pix=None, lse_ws=None, scale=None, stream=None):
+    """Block-energy profiles of the F*H pixel rows of every head: [heads][F*H][nb]
+    (and, with energy=True, the block energies [heads][nb][nb] from the same pass).
+
+    Returns (pix, energy or None)."""
+    heads, n = _bhnd(q)
+    if n != F * H * W:
+        raise ValueError(f"n = {n} is not F*H*W = {F * H * W}")
+    nb = (n + BLOCK - 1) // BLOCK
+    dev = q.device
+    if lse_ws is None:
+        lse_ws = torch.empty((heads, nb * BLOCK), dtype=torch.float32, device=dev)
+    if pix is None:
+        pix = torch.empty((heads, F * H, nb), dtype=torch.float32, device=dev)
+    e = torch.empty((heads, nb, nb), dtype=torch.float32, device=dev) if energy is True else (
+        energy if isinstance(energy, torch.Tensor) else None)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = load().calibatt_pixel_row_energy(_ptr(q), _ptr(k), heads, F, H, W, HEAD_DIM, scale, _ptr(lse_ws), _ptr(e),
+                                          _ptr(pix), _stream(stream))
+    _check(rc, "calibatt_pixel_row_energy")
+    return pix, e
+
+
+def spatial_score(pix, F, H, k_anchor=5, gamma=0.87, score=None, flag=True, stream=None):
+    """Spatial similarity score per head from pixel-row profiles; returns
+    (score fp32 [heads], flag uint8 [heads] or None), flag = score > gamma."""
+    _cuda_tensor(pix, torch.float32, "pix")
+    heads, rows, nb = pix.shape
+    if rows != F * H:
+        raise ValueError(f"pix has {rows} rows per head, not F*H = {F * H}")
+    dev = pix.device
+    if score is None:
+        score = torch.empty((heads,), dtype=torch.float32, device=dev)
+    if flag is True:
+        flag = torch.empty((heads,), dtype=torch.uint8, device=dev)
+    elif flag is False:
+        flag = None
+    rc = load().calibatt_spatial_score(_ptr(pix), heads, F, H, nb, k_anchor, float(gamma), _ptr(score), _ptr(flag),
+                                       _stream(stream))
+    _check(rc, "calibatt_spatial_score")
+    return score, flag
 
 
 def select_mask(energy, eps, mask=True, kept=True, counts=None, stream=None):

@@ -305,6 +305,63 @@ size_t calibatt_aggregate_workspace_size(int heads, int nb) {
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
+int calibatt_pixel_row_energy(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int frames, int H,
+                              int W, int d, float scale, float* lse_ws, float* energy, float* pix_energy,
+                              calibatt_stream_t stream) {
+  if (frames < 1 || H < 1 || W < 1 || !pix_energy) return CALIBATT_ERR_ARG;
+  const int64_t n64 = static_cast<int64_t>(frames) * H * W;
+  if (n64 > INT_MAX / 2) return CALIBATT_ERR_ARG;
+  const int n = static_cast<int>(n64);
+  int rc = check_qkv(q, k, nullptr, nullptr, heads, n, d);
+  if (rc != CALIBATT_OK) return rc;
+  const int nb = (n + 127) / 128;
+  if (nb > CALIBATT_MAX_CALIB_NB) return CALIBATT_ERR_UNSUPPORTED;
+  if (!scale_ok(scale) || !lse_ws) return CALIBATT_ERR_ARG;
+  if (!aligned4(lse_ws) || (energy && !aligned4(energy)) || !aligned4(pix_energy)) return CALIBATT_ERR_ALIGN;
+  KernelParams p = base_params();
+  if (!p.status) return CALIBATT_ERR_CUDA;
+  p.n_q = p.n_k = n;
+  p.nbq = p.nbk = nb;
+  p.heads_q = p.heads_kv = heads;
+  p.n_units = heads * nb;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_out = n;
+  p.lse_ws = lse_ws;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t pix_bytes = static_cast<size_t>(heads) * frames * H * nb * sizeof(float);
+  if (cudaMemsetAsync(pix_energy, 0, pix_bytes, st) != cudaSuccess) return CALIBATT_ERR_CUDA;
+  rc = launch_attention(1, q, n, heads, k, nullptr, n, heads, p, st);
+  if (rc != CALIBATT_OK) return rc;
+  p.energy = energy;
+  p.pix_energy = pix_energy;
+  p.pix_W = W;
+  p.pix_rows = frames * H;
+  p.pix_inv_W = 1.0f / static_cast<float>(W);
+  return launch_attention(2, q, n, heads, k, nullptr, n, heads, p, st);
+}
+
+int calibatt_spatial_score(const float* pix_energy, int heads, int frames, int H, int nb, int k_anchor,
+                           float gamma, float* score, uint8_t* flag, calibatt_stream_t stream) {
+  static_assert(kMaxFrameRows == CALIBATT_MAX_FRAME_ROWS, "frame-row table size");
+  if (!pix_energy || !score || heads < 1 || frames < 1 || H < 1 || nb < 1 || k_anchor < 1 || k_anchor > H ||
+      std::isnan(gamma))
+    return CALIBATT_ERR_ARG;
+  if (H > CALIBATT_MAX_FRAME_ROWS) return CALIBATT_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(heads) * frames * H * nb > (int64_t{1} << 40)) return CALIBATT_ERR_ARG;
+  if (!aligned4(pix_energy) || !aligned4(score)) return CALIBATT_ERR_ALIGN;
+  int32_t anchors[CALIBATT_MAX_FRAME_ROWS];
+  calibatt_anchor_rows(H, k_anchor, anchors);
+  RowAnchorTable tab;
+  for (int r = 0; r < H; ++r) {
+    int best = 0;  // nearest anchor, ties to the lower one
+    for (int j = 1; j < k_anchor; ++j)
+      if (std::abs(r - anchors[j]) < std::abs(r - anchors[best])) best = j;
+    tab.row[r] = anchors[best];
+  }
+  return launch_spatial_score(pix_energy, heads, frames, H, nb, tab, gamma, score, flag,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
 int calibatt_aggregate_masks(const uint16_t* counts, int n_inputs, int heads, int nb, double rho, uint8_t* mask,
                              int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, void* ws,
                              size_t ws_bytes, calibatt_stream_t stream) {

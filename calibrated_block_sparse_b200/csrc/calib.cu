@@ -194,3 +194,76 @@ int launch_gather(const void* q, int n, int heads, const int32_t* rep_heads, int
 }
 
 }  // namespace calibatt
+
+// ------------------------------------------------------------------ spatial score
+// Per head (one CTA): the mean over frames and non-anchor pixel rows r of the
+// cosine similarity between the profile of r and that of its nearest anchor
+// row (explainer §三, the spatial similarity score; §二 observation 4). Warp w
+// takes pixel rows w, w+8, ...; per-warp partial sums are combined in a fixed
+// order, so the score is reproducible for given profiles.
+namespace calibatt {
+namespace {
+
+constexpr int kScoreWarps = 8;
+
+__global__ void __launch_bounds__(kScoreWarps * 32)
+    spatial_score_kernel(const float* __restrict__ pix, int frames, int H, int nb,
+                         const __grid_constant__ RowAnchorTable tab, float gamma, float* score, uint8_t* flag) {
+  const int h = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(frames) * H;
+  const float* base = pix + static_cast<int64_t>(h) * rows * nb;
+  double sum = 0.0;
+  int cnt = 0;
+  for (int64_t R = warp; R < rows; R += kScoreWarps) {
+    const int r = static_cast<int>(R % H);
+    const int a = tab.row[r];
+    if (a == r) continue;  // an anchor row is computed, not copied
+    const float* x = base + R * nb;
+    const float* y = base + (R - r + a) * nb;
+    float xy = 0.f, xx = 0.f, yy = 0.f;
+    for (int c = lane; c < nb; c += 32) {
+      const float xv = __ldg(x + c), yv = __ldg(y + c);
+      xy = fmaf(xv, yv, xy);
+      xx = fmaf(xv, xv, xx);
+      yy = fmaf(yv, yv, yy);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      xy += __shfl_xor_sync(0xffffffffu, xy, o);
+      xx += __shfl_xor_sync(0xffffffffu, xx, o);
+      yy += __shfl_xor_sync(0xffffffffu, yy, o);
+    }
+    sum += (xx > 0.f && yy > 0.f) ? static_cast<double>(xy) / (sqrt(static_cast<double>(xx)) * sqrt(static_cast<double>(yy)))
+                                  : 0.0;
+    ++cnt;
+  }
+  __shared__ double ssum[kScoreWarps];
+  __shared__ int scnt[kScoreWarps];
+  if (lane == 0) {
+    ssum[warp] = sum;
+    scnt[warp] = cnt;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    int c = 0;
+    for (int w = 0; w < kScoreWarps; ++w) {
+      t += ssum[w];
+      c += scnt[w];
+    }
+    const float s = c ? static_cast<float>(t / c) : 1.0f;
+    score[h] = s;
+    if (flag) flag[h] = s > gamma ? 1 : 0;
+  }
+}
+
+}  // namespace
+
+int launch_spatial_score(const float* pix, int heads, int frames, int H, int nb, const RowAnchorTable& tab,
+                         float gamma, float* score, uint8_t* flag, cudaStream_t stream) {
+  spatial_score_kernel<<<heads, kScoreWarps * 32, 0, stream>>>(pix, frames, H, nb, tab, gamma, score, flag);
+  return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
+}
+
+}  // namespace calibatt

@@ -38,11 +38,21 @@ struct KernelParams {
   uint8_t* mask;
   int32_t* kept;
   uint16_t* counts;
+  // pixel-row profiles (energy pass): pix_energy[hq][q / pix_W][c] += ... / pix_W
+  float* pix_energy;   // [heads_q][pix_rows][nbk] or NULL
+  int pix_W, pix_rows;
+  float pix_inv_W;
   int* status;         // device status word
 };
 
 struct AnchorTable {
   int anchor[kMaxAnchors];
+};
+
+// For each row r of a frame, the row of its nearest anchor (spatial score).
+constexpr int kMaxFrameRows = 512;
+struct RowAnchorTable {
+  int32_t row[kMaxFrameRows];
 };
 
 int launch_attention(int mode, const void* q, int q_rows, int q_heads, const void* k, const void* v, int kv_rows,
@@ -56,6 +66,8 @@ int launch_accumulate(const uint8_t* mask, int64_t cells, uint16_t* counts, cuda
 int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold, uint8_t* mask, int32_t* row_ptr,
                      int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* row_cnt, int* status,
                      cudaStream_t stream);
+int launch_spatial_score(const float* pix, int heads, int frames, int H, int nb, const RowAnchorTable& tab,
+                         float gamma, float* score, uint8_t* flag, cudaStream_t stream);
 int launch_gather(const void* q, int n, int heads, const int32_t* rep_heads, int n_rep, int H, int W, int k_anchor,
                   const AnchorTable& tab, void* out, int* status, cudaStream_t stream);
 

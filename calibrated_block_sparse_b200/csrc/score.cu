@@ -267,6 +267,22 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           }
           if (MODE == kLse) l_run += acc;
         }
+        if (MODE == kEnergy && p.pix_energy) {
+          // pixel-row profiles: a segmented scan over the warp's rows (a
+          // pixel row is a run of consecutive lanes), then one atomic add per
+          // pixel row from the run's last lane
+          const int key = row_valid ? qrow / p.pix_W : -1;
+          float v = acc;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float vu = __shfl_up_sync(0xffffffffu, v, o);
+            const int ku = __shfl_up_sync(0xffffffffu, key, o);
+            if (lane >= o && ku == key) v += vu;
+          }
+          const int kn = __shfl_down_sync(0xffffffffu, key, 1);
+          if (ok && key >= 0 && (lane == 31 || kn != key))
+            atomicAdd(p.pix_energy + (static_cast<int64_t>(u.hq) * p.pix_rows + key) * p.nbk + j, v * p.pix_inv_W);
+        }
         if (MODE == kEnergy) {
           // this warp's share of E[r][j]: sum over its 32 rows
 #pragma unroll

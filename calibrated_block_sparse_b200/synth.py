@@ -15,6 +15,9 @@ attention inputs of those models at the same shapes):
   zero-padded to d = 128. w_m ~ N(0, sigma_h^2 I_3) and b_m ~ U[0, 2 pi) are
   drawn per head only, fixed across inputs, which is what makes the block
   structure stable from one input to the next;
+* the workload's spatially repeated heads attend across frames, alike for
+  every pixel row of a frame (the pages' observation 4): their features
+  ignore the row, w_m[1] = 0, so e depends on (f/F, c/W) only;
 * values are rounded to bf16 (round to nearest even).
 """
 from __future__ import annotations
@@ -98,6 +101,8 @@ def fourier_features(wl: Workload, head: int) -> torch.Tensor:
     rng = np.random.default_rng(_seed(wl.config_id, 11, head))
     sigma = head_sigma(wl, head)
     w = rng.normal(0.0, sigma, size=(N_FEAT, 3))
+    if head in wl.repeat_heads:
+        w[:, 1] = 0.0  # no dependence on the pixel row
     b = rng.uniform(0.0, 2.0 * math.pi, size=(N_FEAT,))
     pos = positions(wl.F, wl.H, wl.W)
     e = np.cos(2.0 * math.pi * pos @ w.T + b)

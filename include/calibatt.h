@@ -196,6 +196,45 @@ int calibatt_aggregate_masks(const uint16_t* counts, int n_inputs, int heads, in
                              int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, void* ws,
                              size_t ws_bytes, calibatt_stream_t stream);
 
+/* ---------------------------------------------------------------- spatial repetition */
+
+/* Largest frame height H accepted by calibatt_spatial_score. */
+#define CALIBATT_MAX_FRAME_ROWS 512
+
+/* Block-energy profiles of pixel rows (explainer §二 observation 4 and §六:
+ * the pixel rows of a frame attend alike; §三: the spatial similarity score
+ * is computed per head at calibration). Tokens are frame-major, row-major
+ * inside a frame (token = f*H*W + r*W + c, n = frames*H*W); pixel row
+ * R = f*H + r holds W queries. With P = softmax(scale * Q K^T) over all n keys,
+ *   pix_energy[h][R][c] = (1 / W) * sum_{i in pixel row R, j in key block c} P_ij.
+ * Two passes as in calibatt_block_energy: the first writes the row
+ * log-sum-exp to lse_ws, the second recomputes S; when `energy` is not NULL
+ * that pass also writes the block energies of calibatt_block_energy (no
+ * selection). pix_energy is cleared first and then accumulated with fp32
+ * atomics, so its last bits may differ between runs.
+ *   lse_ws     : device fp32 scratch [heads][nb*128]
+ *   energy     : device fp32 [heads][nb][nb] or NULL
+ *   pix_energy : device fp32 [heads][frames*H][nb] (output)
+ * Requires nb <= CALIBATT_MAX_CALIB_NB. */
+int calibatt_pixel_row_energy(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int frames, int H,
+                              int W, int d, float scale, float* lse_ws, float* energy, float* pix_energy,
+                              calibatt_stream_t stream);
+
+/* Spatial similarity score of each head (explainer §三: a head is marked
+ * spatially repeated when its score exceeds gamma = 0.87; the pages give no
+ * formula). Reading used: the mean, over every frame and every pixel row r
+ * that is not an anchor row, of the cosine similarity between the profile of
+ * row r and the profile of its nearest anchor row (calibatt_anchor_rows; ties
+ * -> lower anchor), i.e. the row whose output a repeated head copies to r.
+ * A cosine with an all-zero profile counts as 0; with k_anchor = H the score
+ * is 1.
+ *   pix_energy : device fp32 [heads][frames*H][nb] (calibatt_pixel_row_energy)
+ *   score      : device fp32 [heads] (output)
+ *   flag       : device uint8 [heads] or NULL (output: score > gamma)
+ * Requires 1 <= k_anchor <= H <= CALIBATT_MAX_FRAME_ROWS. */
+int calibatt_spatial_score(const float* pix_energy, int heads, int frames, int H, int nb, int k_anchor,
+                           float gamma, float* score, uint8_t* flag, calibatt_stream_t stream);
+
 /* ---------------------------------------------------------------- no-allocation variant */
 
 /* Largest heads * nb accepted by calibatt_aggregate_masks_noalloc. */

@@ -138,6 +138,18 @@ def test_argument_errors_are_caught_on_the_host(binding):
     assert lib.calibatt_aggregate_masks(fake, 4, 1, 16, 0.5, fake, fake, fake, 256, fake, fake, 4, None) == -1
     assert lib.calibatt_aggregate_masks(fake, 0, 1, 16, 0.5, fake, fake, fake, 256, fake, fake, 1024, None) == -1
     assert lib.calibatt_accumulate_masks(None, 10, fake, None) == -1
+    # pixel-row profiles and the spatial score
+    odd2 = P(0x100002)       # 2-byte aligned only
+    assert lib.calibatt_pixel_row_energy(fake, fake, 1, 0, 8, 16, 128, 0.1, fake, None, fake, None) == -1
+    assert lib.calibatt_pixel_row_energy(fake, fake, 1, 2, 8, 16, 64, 0.1, fake, None, fake, None) == -4
+    assert lib.calibatt_pixel_row_energy(fake, fake, 1, 1025, 8, 16, 128, 0.1, fake, None, fake, None) == -4
+    assert lib.calibatt_pixel_row_energy(fake, fake, 1, 2, 8, 16, 128, 0.1, fake, None, None, None) == -1
+    assert lib.calibatt_pixel_row_energy(fake, fake, 1, 2, 8, 16, 128, 0.1, fake, None, odd2, None) == -3
+    assert lib.calibatt_spatial_score(fake, 1, 2, 600, 16, 5, 0.87, fake, None, None) == -4
+    assert lib.calibatt_spatial_score(fake, 1, 2, 4, 16, 5, 0.87, fake, None, None) == -1
+    assert lib.calibatt_spatial_score(fake, 1, 2, 8, 16, 5, float("nan"), fake, None, None) == -1
+    assert lib.calibatt_spatial_score(fake, 1, 2, 8, 16, 5, 0.87, None, None, None) == -1
+    assert lib.calibatt_spatial_score(odd2, 1, 2, 8, 16, 5, 0.87, fake, None, None) == -3
 
 
 def test_workspace_sizes(binding):

@@ -11,10 +11,15 @@ benchmark times, on sampled outputs the fp64 oracle computes one by one.
   heads (k = 5 of 30 rows) on sampled rows.
 * Calibration sweep at the Wan-720p shape: eps in {0.84, 0.9, 0.95, 0.99} on
   sampled block-rows; aggregation of 16 inputs against the oracle aggregator.
+* Spatial repetition at the Wan-720p and Mochi shapes: pixel-row profiles and
+  scores of every head; the heads flagged at gamma = 0.87 are the workloads'
+  repeated heads.
 
 Inputs come from the seeded generator (synth), drawn on the device; the
 sampled heads are copied to the host for the oracle.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -177,3 +182,32 @@ def test_mochi_calibrated_attention_sampled_rows(oracle):
         og = o[h].float().cpu().numpy().astype(np.float64)[rows]
         ok, err, bound = attn_tolerance_ok(og, o_ref)
         assert ok, (h, err, bound)
+
+
+@pytest.mark.parametrize("name", ["wan720", "mochi480"])
+def test_spatial_classification_full_size(oracle, name):
+    """Pixel-row profiles and spatial scores of every head: the flagged heads
+    (score > 0.87) are exactly the workload's repeated heads; sampled profile
+    rows against the oracle; every score against the oracle's score of the
+    same profiles."""
+    binding = require_gpu()
+    wl = synth.WORKLOADS[name]
+    dev = torch.device(DEV)
+    q, k, _ = synth.qkv(wl, 0, device=dev, with_v=False)
+    pix, _ = binding.pixel_row_energy(q, k, wl.F, wl.H, wl.W)
+    s, flag = binding.spatial_score(pix, wl.F, wl.H, wl.k_anchor, gamma=0.87)
+    assert binding.get_status() == 0
+    assert np.nonzero(flag.cpu().numpy())[0].tolist() == list(wl.repeat_heads)
+    got = pix.cpu().numpy().astype(np.float64)
+    s = s.cpu().numpy()
+    for h in range(wl.heads):
+        assert abs(s[h] - oracle.spatial_score(got[h], wl.F, wl.H, wl.k_anchor)) <= 1e-5
+    rows_per_head = wl.F * wl.H
+    heads = [0, wl.repeat_heads[0]]
+    sample = np.array([h * rows_per_head + r for h in heads for r in (0, rows_per_head - 1)], np.int64)
+    hs = sorted(set(heads))
+    ref = oracle.pixel_row_energy(_bits(q[hs].cpu()), _bits(k[hs].cpu()), wl.F, wl.H, wl.W,
+                                  prows=np.array([hs.index(int(g // rows_per_head)) * rows_per_head +
+                                                  int(g % rows_per_head) for g in sample], np.int64),
+                                  threads=min(16, os.cpu_count() or 1))
+    assert _energy_ok(got.reshape(-1, got.shape[-1])[sample], ref)
