@@ -428,6 +428,24 @@ def run_ours(args, world, rank, local):
 
         with torch.cuda.stream(gstream):
             a_ms = graph_time(agg_call, 20, gstream)
+        # spatial repetition: pixel-row profiles (same two passes, plus the
+        # profile atomics) and the per-head score
+        pix = torch.empty((ch, wl.F * wl.H, nb), dtype=torch.float32, device=dev)
+
+        def pix_call():
+            binding.pixel_row_energy(qc, kc, wl.F, wl.H, wl.W, pix=pix, lse_ws=lse_ws, stream=stream)
+
+        pix_call()
+        p_ms = cuda_time(pix_call, 2, stream)
+        sscore = torch.empty(ch, dtype=torch.float32, device=dev)
+        sflag = torch.empty(ch, dtype=torch.uint8, device=dev)
+
+        def score_call():
+            binding.spatial_score(pix, wl.F, wl.H, wl.k_anchor, score=sscore, flag=sflag,
+                                  stream=torch.cuda.current_stream())
+
+        with torch.cuda.stream(gstream):
+            sc_ms = graph_time(score_call, 20, gstream)
         binding.check_status(what="calibration")
         kept_agg = int(annz.item())
         agg_bytes = ch * nb * nb * (2 + 1 + 1) + kept_agg * 4 + (ch * nb + 1) * 4 * 3
@@ -438,8 +456,12 @@ def run_ours(args, world, rank, local):
             "select_ms": s_ms, "select_gbs": sel_bytes / (s_ms * 1e-3) / 1e9,
             "aggregate_ms": a_ms, "aggregate_gbs": agg_bytes / (a_ms * 1e-3) / 1e9,
             "eps": 0.9, "kept_fraction_at_eps": float(cmask.float().mean().item()),
+            "pixel_row_energy_ms": p_ms, "pixel_row_energy_tflops_issued": f_energy_issued / (p_ms * 1e-3) / 1e12,
+            "spatial_score_ms": sc_ms,
+            "spatial_score_gbs": ch * wl.F * (wl.H - wl.k_anchor) * nb * 8 / (sc_ms * 1e-3) / 1e9,
+            "spatial_flagged_heads": np.nonzero(sflag.cpu().numpy())[0].tolist(),
         }
-        del qc, kc, lse_ws, energy, cmask, ccounts
+        del qc, kc, lse_ws, energy, cmask, ccounts, pix
 
     # ---- roofline of the dominant kernel (the block-sparse attention kernel)
     pk, pk_src = peaks()
