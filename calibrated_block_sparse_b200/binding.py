@@ -69,6 +69,9 @@ def load(build_if_missing: bool = False):
             "calibatt_aggregate_masks": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P, sz, P]),
             "calibatt_aggregate_masks_noalloc": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P]),
             "calibatt_pixel_row_energy": (i32, [P, P, i32, i32, i32, i32, i32, f32, P, P, P, P]),
+            "calibatt_build_mixed_plan": (i32, [P, i32, i32, P, i32, P, i32, i32, i32, i32, P, P]),
+            "calibatt_mixed_attn_fwd": (i32, [P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, i64, P, i32, P, i32,
+                                              P, P, P, sz, P]),
             "calibatt_spatial_score": (i32, [P, i32, i32, i32, i32, i32, f32, P, P, P]),
         }
         for name, (res, args) in sig.items():
@@ -144,6 +147,20 @@ def build_plan(row_ptr: np.ndarray, heads: int, nb: int, head_active=None) -> np
     return out[: int(n[0])].copy()
 
 
+def build_mixed_plan(row_ptr: np.ndarray, heads: int, nb: int, rep_heads, F: int, H: int, W: int,
+                     k_anchor: int = 5) -> np.ndarray:
+    """Work list of the block-sparse units of the heads not in rep_heads and
+    the anchor-query units of the repeated heads, head by head."""
+    rp = np.ascontiguousarray(row_ptr, np.int32)
+    rep = np.ascontiguousarray([int(h) for h in rep_heads], np.int32)
+    nbq_b = -(-F * k_anchor * W // BLOCK)
+    out = np.empty(heads * nb + len(rep) * nbq_b, np.int32)
+    n = np.zeros(1, np.int32)
+    _check(load().calibatt_build_mixed_plan(_ptr(rp), heads, nb, None, len(rep), _ptr(rep) if len(rep) else None,
+                                            F, H, W, k_anchor, _ptr(out), _ptr(n)), "build_mixed_plan")
+    return out[: int(n[0])].copy()
+
+
 def anchor_rows(H: int, k_anchor: int) -> np.ndarray:
     out = np.empty(k_anchor, np.int32)
     _check(load().calibatt_anchor_rows(H, k_anchor, _ptr(out)), "anchor_rows")
@@ -202,6 +219,34 @@ def repeat_attn_fwd(q, k, v, F, H, W, rep_heads, k_anchor=5, o=None, lse=None, w
                                          _ptr(rep_heads), n_rep, _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
                                          _stream(stream))
     _check(rc, "calibatt_repeat_attn_fwd")
+    return o, lse
+
+
+def mixed_attn_fwd(q, k, v, F, H, W, row_ptr, col_idx, rep_heads, work_list, k_anchor=5, o=None, lse=None,
+                   ws=None, scale=None, want_lse=True, stream=None):
+    """Block-sparse and repeated heads in one persistent launch; returns (o, lse)."""
+    heads, n = _bhnd(q)
+    _bhnd(k, "k")
+    _bhnd(v, "v")
+    _cuda_tensor(row_ptr, torch.int32, "row_ptr")
+    _cuda_tensor(col_idx, torch.int32, "col_idx")
+    _cuda_tensor(rep_heads, torch.int32, "rep_heads")
+    _cuda_tensor(work_list, torch.int32, "work_list")
+    n_rep = rep_heads.numel()
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((heads, n), dtype=torch.float32, device=q.device)
+    if ws is None and n_rep > 0:
+        ws = torch.empty(repeat_workspace_size(n_rep, F, H, W, k_anchor), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = load().calibatt_mixed_attn_fwd(_ptr(q), _ptr(k), _ptr(v), heads, F, H, W, HEAD_DIM, k_anchor, scale,
+                                        _ptr(row_ptr), _ptr(col_idx) if col_idx.numel() else None, col_idx.numel(),
+                                        _ptr(rep_heads) if n_rep else None, n_rep,
+                                        _ptr(work_list) if work_list.numel() else None, work_list.numel(),
+                                        _ptr(o), _ptr(lse), _ptr(ws), ws.numel() if ws is not None else 0,
+                                        _stream(stream))
+    _check(rc, "calibatt_mixed_attn_fwd")
     return o, lse
 
 

@@ -63,6 +63,36 @@ KernelParams base_params() {
   return p;
 }
 
+
+// Anchor-query segment of the attention kernel for n_rep repeated heads: the
+// packed anchor queries (calibatt_repeat_workspace_size layout), the band of
+// rows each anchor row is broadcast to (nearest anchor, ties to the lower
+// one), and the anchor rows for the gather.
+void set_repeat_segment(KernelParams& p, int frames, int H, int W, int k_anchor, int n_rep, const int32_t* rep_heads,
+                        AnchorTable& tab) {
+  int32_t anchors[kMaxAnchors];
+  calibatt_anchor_rows(H, k_anchor, anchors);
+  for (int j = 0; j < k_anchor; ++j) {
+    p.band_lo[j] = INT_MAX;
+    p.band_hi[j] = 0;
+    tab.anchor[j] = anchors[j];
+  }
+  for (int r = 0; r < H; ++r) {
+    int best = 0;
+    for (int j = 1; j < k_anchor; ++j)
+      if (std::abs(r - anchors[j]) < std::abs(r - anchors[best])) best = j;
+    p.band_lo[best] = std::min(p.band_lo[best], r);
+    p.band_hi[best] = std::max(p.band_hi[best], r + 1);
+  }
+  p.n_q_b = frames * k_anchor * W;
+  p.nbq_b = (p.n_q_b + 127) / 128;
+  p.heads_q_b = n_rep;
+  p.head_map_b = rep_heads;
+  p.rep_H = H;
+  p.rep_W = W;
+  p.rep_k = k_anchor;
+}
+
 }  // namespace
 }  // namespace calibatt
 
@@ -122,19 +152,21 @@ int calibatt_build_plan(const int32_t* row_ptr, int heads, int nb, const uint8_t
                         int32_t* n_work) {
   if (!row_ptr || !work_list || !n_work || heads < 1 || nb < 1) return CALIBATT_ERR_ARG;
   if (static_cast<int64_t>(heads) * nb > INT_MAX / 2) return CALIBATT_ERR_ARG;
-  std::vector<int32_t> units;
-  units.reserve(static_cast<size_t>(heads) * nb);
+  int32_t* out = work_list;
+  std::vector<int32_t> units(static_cast<size_t>(nb));
   for (int h = 0; h < heads; ++h) {
     if (head_active && !head_active[h]) continue;
-    for (int r = 0; r < nb; ++r) units.push_back(h * nb + r);
+    for (int r = 0; r < nb; ++r) {
+      units[r] = h * nb + r;
+      if (row_ptr[units[r] + 1] < row_ptr[units[r]]) return CALIBATT_ERR_CSR;
+    }
+    // longest first within the head; equal counts keep block order
+    std::stable_sort(units.begin(), units.end(), [&](int32_t a, int32_t b) {
+      return (row_ptr[a + 1] - row_ptr[a]) > (row_ptr[b + 1] - row_ptr[b]);
+    });
+    out = std::copy(units.begin(), units.end(), out);
   }
-  for (int32_t u : units)
-    if (row_ptr[u + 1] < row_ptr[u]) return CALIBATT_ERR_CSR;
-  std::stable_sort(units.begin(), units.end(), [&](int32_t a, int32_t b) {
-    return (row_ptr[a + 1] - row_ptr[a]) > (row_ptr[b + 1] - row_ptr[b]);
-  });
-  std::copy(units.begin(), units.end(), work_list);
-  *n_work = static_cast<int32_t>(units.size());
+  *n_work = static_cast<int32_t>(out - work_list);
   return CALIBATT_OK;
 }
 
@@ -185,6 +217,85 @@ int calibatt_sparse_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, con
   return launch_attention(0, q, n, heads, k, v, n, heads, p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int calibatt_build_mixed_plan(const int32_t* row_ptr, int heads, int nb, const uint8_t* head_active, int n_rep,
+                              const int32_t* rep_heads, int frames, int H, int W, int k_anchor, int32_t* work_list,
+                              int32_t* n_work) {
+  if (!row_ptr || !work_list || !n_work || heads < 1 || nb < 1 || n_rep < 0 || n_rep > heads ||
+      (n_rep > 0 && !rep_heads) || frames < 1 || H < 1 || W < 1 || k_anchor < 1 || k_anchor > H)
+    return CALIBATT_ERR_ARG;
+  const int64_t nbq_b = (static_cast<int64_t>(frames) * k_anchor * W + 127) / 128;
+  if (static_cast<int64_t>(heads) * nb + n_rep * nbq_b > INT_MAX / 2) return CALIBATT_ERR_ARG;
+  for (int i = 0; i < n_rep; ++i)
+    if (rep_heads[i] < 0 || rep_heads[i] >= heads) return CALIBATT_ERR_ARG;
+  int32_t* out = work_list;
+  // first the repeated heads' anchor-query units (each takes every key block)
+  for (int i = 0; i < n_rep; ++i)
+    for (int64_t b = 0; b < nbq_b; ++b) *out++ = static_cast<int32_t>(heads * nb + i * nbq_b + b);
+  std::vector<int32_t> units(static_cast<size_t>(nb));
+  for (int h = 0; h < heads; ++h) {
+    bool repeated = false;
+    for (int i = 0; i < n_rep; ++i) repeated = repeated || rep_heads[i] == h;
+    if (repeated || (head_active && !head_active[h])) continue;
+    for (int r = 0; r < nb; ++r) {
+      units[r] = h * nb + r;
+      if (row_ptr[units[r] + 1] < row_ptr[units[r]]) return CALIBATT_ERR_CSR;
+    }
+    std::stable_sort(units.begin(), units.end(), [&](int32_t a, int32_t b) {
+      return (row_ptr[a + 1] - row_ptr[a]) > (row_ptr[b + 1] - row_ptr[b]);
+    });
+    out = std::copy(units.begin(), units.end(), out);
+  }
+  *n_work = static_cast<int32_t>(out - work_list);
+  return CALIBATT_OK;
+}
+
+int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v, int heads,
+                            int frames, int H, int W, int d, int k_anchor, float scale, const int32_t* row_ptr,
+                            const int32_t* col_idx, int64_t nnz, const int32_t* rep_heads, int32_t n_rep,
+                            const int32_t* work_list, int32_t n_work, calibatt_bf16* o, float* lse, void* ws,
+                            size_t ws_bytes, calibatt_stream_t stream) {
+  if (!v || !o || frames < 1 || H < 1 || W < 1) return CALIBATT_ERR_ARG;
+  const int64_t n64 = static_cast<int64_t>(frames) * H * W;
+  if (n64 > INT_MAX / 2) return CALIBATT_ERR_ARG;
+  const int n = static_cast<int>(n64);
+  int rc = check_qkv(q, k, v, o, heads, n, d);
+  if (rc != CALIBATT_OK) return rc;
+  if (k_anchor < 1 || k_anchor > H) return CALIBATT_ERR_ARG;
+  if (k_anchor > kMaxAnchors) return CALIBATT_ERR_UNSUPPORTED;
+  const int nb = (n + 127) / 128;
+  const int64_t nbq_b = (static_cast<int64_t>(frames) * k_anchor * W + 127) / 128;
+  if (!scale_ok(scale) || !row_ptr || nnz < 0 || (nnz > 0 && !col_idx) || n_rep < 0 || n_rep > heads ||
+      (n_rep > 0 && !rep_heads) || n_work < 0 ||
+      static_cast<int64_t>(n_work) > static_cast<int64_t>(heads) * nb + n_rep * nbq_b ||
+      (n_work > 0 && !work_list))
+    return CALIBATT_ERR_ARG;
+  if (n_rep > 0 && (!ws || ws_bytes < calibatt_repeat_workspace_size(n_rep, frames, H, W, k_anchor)))
+    return CALIBATT_ERR_ARG;
+  if ((n_rep > 0 && !aligned16(ws)) || (lse && !aligned4(lse))) return CALIBATT_ERR_ALIGN;
+  KernelParams p = base_params();
+  if (!p.status) return CALIBATT_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (n_rep > 0) {
+    AnchorTable tab;
+    set_repeat_segment(p, frames, H, W, k_anchor, n_rep, rep_heads, tab);
+    rc = launch_gather(q, n, heads, rep_heads, n_rep, H, W, k_anchor, tab, ws, p.status, st);
+    if (rc != CALIBATT_OK) return rc;
+  }
+  p.n_q = p.n_k = n;
+  p.nbq = p.nbk = nb;
+  p.heads_q = p.heads_kv = heads;
+  p.n_units = n_work;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.work_list = work_list;
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.nnz = nnz;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.n_out = n;
+  return launch_attention(0, q, n, heads, k, v, n, heads, p, st, n_rep > 0 ? ws : nullptr, p.n_q_b, n_rep);
+}
+
 size_t calibatt_repeat_workspace_size(int n_rep, int frames, int H, int W, int k_anchor) {
   if (n_rep < 1 || frames < 1 || H < 1 || W < 1 || k_anchor < 1) return 0;
   const size_t bytes = static_cast<size_t>(n_rep) * frames * k_anchor * W * 128 * 2;
@@ -208,45 +319,22 @@ int calibatt_repeat_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, con
   if (!ws || ws_bytes < calibatt_repeat_workspace_size(n_rep, frames, H, W, k_anchor)) return CALIBATT_ERR_ARG;
   if (!aligned16(ws) || (lse && !aligned4(lse))) return CALIBATT_ERR_ALIGN;
 
-  int32_t anchors[kMaxAnchors];
-  calibatt_anchor_rows(H, k_anchor, anchors);
   KernelParams p = base_params();
   if (!p.status) return CALIBATT_ERR_CUDA;
-  // nearest anchor of every row (ties to the lower anchor) -> contiguous bands
-  for (int j = 0; j < k_anchor; ++j) {
-    p.band_lo[j] = INT_MAX;
-    p.band_hi[j] = 0;
-  }
-  for (int r = 0; r < H; ++r) {
-    int best = 0;
-    for (int j = 1; j < k_anchor; ++j)
-      if (std::abs(r - anchors[j]) < std::abs(r - anchors[best])) best = j;
-    p.band_lo[best] = std::min(p.band_lo[best], r);
-    p.band_hi[best] = std::max(p.band_hi[best], r + 1);
-  }
   AnchorTable tab;
-  for (int j = 0; j < k_anchor; ++j) tab.anchor[j] = anchors[j];
-
+  set_repeat_segment(p, frames, H, W, k_anchor, n_rep, rep_heads, tab);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int n_anchor = frames * k_anchor * W;
   rc = launch_gather(q, n, heads, rep_heads, n_rep, H, W, k_anchor, tab, ws, p.status, st);
   if (rc != CALIBATT_OK) return rc;
-  p.n_q = n_anchor;
   p.n_k = n;
-  p.nbq = (n_anchor + 127) / 128;
   p.nbk = (n + 127) / 128;
-  p.heads_q = n_rep;
   p.heads_kv = heads;
-  p.n_units = n_rep * p.nbq;
+  p.n_units = n_rep * p.nbq_b;  // every unit is an anchor-query unit (no first segment)
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.head_map = rep_heads;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.n_out = n;
-  p.rep_H = H;
-  p.rep_W = W;
-  p.rep_k = k_anchor;
-  return launch_attention(0, ws, n_anchor, n_rep, k, v, n, heads, p, st);
+  return launch_attention(0, ws, p.n_q_b, n_rep, k, v, n, heads, p, st, ws, p.n_q_b, n_rep);
 }
 
 int calibatt_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int n, int d, float scale,

@@ -61,8 +61,9 @@ struct AttnLayout {
 };
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ KernelParams p) {
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qb,
+                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const __grid_constant__ KernelParams p) {
   using L = AttnLayout;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 8 && lane == 0) {
     // ---------------------------------------------------------- TMA producer
     tma_prefetch_desc(&tm_q);
+    if (p.nbq_b > 0) tma_prefetch_desc(&tm_qb);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     Cursor cur[2];
@@ -125,9 +127,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (c.j == 0) {
         if (!mbar_wait(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status)) return false;
         uint8_t* dst = smem + L::kQOff + s * kTile;
+        const CUtensorMap* qmap = c.u.rep ? &tm_qb : &tm_q;
         mbar_arrive_expect_tx(&bar.q_full[s], kTile);
-        tma_load_3d(dst, &tm_q, &bar.q_full[s], 0, c.u.r * 128, c.u.hq);
-        tma_load_3d(dst + kHalf, &tm_q, &bar.q_full[s], 64, c.u.r * 128, c.u.hq);
+        tma_load_3d(dst, qmap, &bar.q_full[s], 0, c.u.r * 128, c.u.hq);
+        tma_load_3d(dst + kHalf, qmap, &bar.q_full[s], 64, c.u.r * 128, c.u.hq);
         ++n_q[s];
       }
       return load_tile(&tm_k, block_col(p, c.u, c.j), c.u.hkv);
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!load_unit(p, unit_index(g, G, round), u)) break;
       if (!u.write) continue;
       const int qrow = u.r * 128 + row;
-      const bool row_valid = qrow < p.n_q;
+      const bool row_valid = qrow < (u.rep ? p.n_q_b : p.n_q);
       if (u.nnz == 0) {
         // no kept block: O = 0, lse = -inf
         if (row_valid) {
@@ -326,7 +329,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int64_t dst0 = 0;
       int n_dst = 0, dst_stride = 0;
       if (row_valid) {
-        if (p.rep_W > 0) {
+        if (u.rep) {
           const int kw = p.rep_k * p.rep_W;
           const int f = qrow / kw, rem = qrow % kw;
           const int ja = rem / p.rep_W, c = rem % p.rep_W;
@@ -369,8 +372,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const KernelParams& p,
-                cudaStream_t stream) {
+int launch_attn(const CUtensorMap& mq, const CUtensorMap& mqb, const CUtensorMap& mk, const CUtensorMap& mv,
+                const KernelParams& p, cudaStream_t stream) {
   static_assert(AttnLayout::kDynSmem <= 232448, "shared memory budget");
   static bool configured = false;  // per process; the attribute is per function
   if (!configured) {
@@ -383,21 +386,23 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
   int grid = (p.n_units + 1) / 2;
   const int sms = sm_count();
   if (grid > sms) grid = sms;
-  attn_kernel<<<grid, kAttnThreads, AttnLayout::kDynSmem, stream>>>(mq, mk, mv, p);
+  attn_kernel<<<grid, kAttnThreads, AttnLayout::kDynSmem, stream>>>(mq, mqb, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
 }
 
 }  // namespace
 
 int launch_attention(int mode, const void* q, int q_rows, int q_heads, const void* k, const void* v, int kv_rows,
-                     int kv_heads, const KernelParams& p, cudaStream_t stream) {
-  CUtensorMap mq, mk, mv;
+                     int kv_heads, const KernelParams& p, cudaStream_t stream, const void* qb, int qb_rows,
+                     int qb_heads) {
+  CUtensorMap mq, mqb, mk, mv;
   int rc = make_map(&mq, q, q_rows, q_heads);
+  if (rc == CALIBATT_OK) rc = qb ? make_map(&mqb, qb, qb_rows, qb_heads) : (mqb = mq, CALIBATT_OK);
   if (rc == CALIBATT_OK) rc = make_map(&mk, k, kv_rows, kv_heads);
   if (rc == CALIBATT_OK && mode == kAttn) rc = make_map(&mv, v, kv_rows, kv_heads);
   if (rc != CALIBATT_OK) return rc;
   switch (mode) {
-    case kAttn: return launch_attn(mq, mk, mv, p, stream);
+    case kAttn: return launch_attn(mq, mqb, mk, mv, p, stream);
     case kLse:
     case kEnergy: return launch_score(mode, mq, mk, p, stream);
     default: return CALIBATT_ERR_ARG;

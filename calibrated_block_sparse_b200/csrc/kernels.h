@@ -26,8 +26,14 @@ struct KernelParams {
   __nv_bfloat16* o;          // output [heads_kv][n_out][128]
   float* lse;                // output [heads_kv][n_out] or NULL
   int64_t n_out;             // rows per head of o / lse
+  // Second unit segment (attention only): anchor-query units of spatially
+  // repeated heads, unit codes heads_q*nbq .. + heads_q_b*nbq_b - 1. Their Q
+  // rows come from the packed anchor tensor (n_q_b rows per head), they take
+  // every key block, and head_map_b gives their K/V/O head. nbq_b = 0: none.
+  int n_q_b, nbq_b, heads_q_b;
+  const int32_t* head_map_b;
   // repeated heads: a packed anchor query q = f*(k*W) + j*W + c writes rows
-  // band_lo[j] .. band_hi[j]-1 of frame f, column c (rep_W = 0: off)
+  // band_lo[j] .. band_hi[j]-1 of frame f, column c
   int rep_H, rep_W, rep_k;
   int band_lo[kMaxAnchors], band_hi[kMaxAnchors];
   // energy passes
@@ -55,8 +61,11 @@ struct RowAnchorTable {
   int32_t row[kMaxFrameRows];
 };
 
+// qb: the packed anchor tensor of the second unit segment ([qb_heads][qb_rows][128])
+// or NULL.
 int launch_attention(int mode, const void* q, int q_rows, int q_heads, const void* k, const void* v, int kv_rows,
-                     int kv_heads, const KernelParams& p, cudaStream_t stream);
+                     int kv_heads, const KernelParams& p, cudaStream_t stream, const void* qb = nullptr,
+                     int qb_rows = 0, int qb_heads = 0);
 
 long long eps_to_fixed(double eps);
 

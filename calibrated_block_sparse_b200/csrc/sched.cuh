@@ -22,12 +22,13 @@ enum Mode : int { kAttn = 0, kLse = 1, kEnergy = 2 };
 
 // ------------------------------------------------------------------ work units
 struct Unit {
-  int hq;      // head index in the Q tensor
+  int hq;      // head index in the Q tensor (second segment: in the anchor tensor)
   int hkv;     // head index in K / V / O
   int r;       // query block
   int nnz;     // kept key blocks
   int base;    // offset into col_idx
   bool write;  // false: malformed work-list entry, produce nothing
+  bool rep;    // second segment: anchor queries of a repeated head
 };
 
 // Static longest-first schedule: the work list is sorted by kept blocks,
@@ -39,21 +40,43 @@ __device__ __forceinline__ int unit_index(int g, int G, int round) {
 __device__ __forceinline__ bool load_unit(const KernelParams& p, int idx, Unit& u) {
   if (idx >= p.n_units) return false;
   int code = p.work_list ? __ldg(p.work_list + idx) : idx;
+  const int n_a = p.heads_q * p.nbq;
   u.write = true;
-  if (code < 0 || code >= p.heads_q * p.nbq) {
+  u.rep = false;
+  if (code >= n_a && p.nbq_b > 0 && code - n_a < p.heads_q_b * p.nbq_b) {
+    // anchor-query unit: every key block, K/V/O head from head_map_b
+    const int c = code - n_a;
+    u.rep = true;
+    u.hq = c / p.nbq_b;
+    u.r = c % p.nbq_b;
+    u.hkv = __ldg(p.head_map_b + u.hq);
+    if (u.hkv < 0 || u.hkv >= p.heads_kv) {
+      record_error(p.status, CALIBATT_ERR_ARG);
+      u.write = false;
+      u.hkv = 0;
+    }
+    u.base = 0;
+    u.nnz = u.write ? p.nbk : 0;
+    return true;
+  }
+  if (code < 0 || code >= n_a) {
     record_error(p.status, CALIBATT_ERR_CSR);
     u.write = false;
     code = 0;
   }
-  u.hq = code / p.nbq;
-  u.r = code % p.nbq;
+  const int nbq = p.nbq > 0 ? p.nbq : 1;
+  u.hq = code / nbq;
+  u.r = code % nbq;
   u.hkv = p.head_map ? __ldg(p.head_map + u.hq) : u.hq;
   if (u.hkv < 0 || u.hkv >= p.heads_kv) {
     record_error(p.status, CALIBATT_ERR_ARG);
     u.write = false;
     u.hkv = 0;
   }
-  if (p.row_ptr) {
+  if (!u.write) {
+    u.base = 0;
+    u.nnz = 0;
+  } else if (p.row_ptr) {
     const int a = __ldg(p.row_ptr + code), b = __ldg(p.row_ptr + code + 1);
     if (a < 0 || b < a || static_cast<int64_t>(b) > p.nnz) {
       record_error(p.status, CALIBATT_ERR_CSR);
@@ -67,13 +90,12 @@ __device__ __forceinline__ bool load_unit(const KernelParams& p, int idx, Unit& 
     u.base = 0;
     u.nnz = p.nbk;
   }
-  if (!u.write) u.nnz = 0;
   return true;
 }
 
 // Key block of the j-th kept tile; out-of-range entries are clamped and reported.
 __device__ __forceinline__ int block_col(const KernelParams& p, const Unit& u, int j) {
-  if (!p.col_idx) return j;
+  if (!p.col_idx || u.rep) return j;
   int c = __ldg(p.col_idx + u.base + j);
   if (c < 0 || c >= p.nbk) {
     record_error(p.status, CALIBATT_ERR_CSR);

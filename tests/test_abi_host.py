@@ -85,18 +85,21 @@ def test_validate_csr(binding, oracle):
     assert binding.validate_csr(rp2, ci, 2, 9) == -2
 
 
-def test_build_plan_is_longest_first(binding, oracle):
+def test_build_plan_is_head_by_head_longest_first(binding, oracle):
     rng = np.random.default_rng(2)
     mask = (rng.random((3, 7, 7)) < rng.random((3, 1, 1))).astype(np.uint8)
     rp, _ = oracle.mask_to_csr(mask)
     work = binding.build_plan(rp, 3, 7)
     nnz = np.diff(rp)
     assert sorted(work.tolist()) == list(range(21))
-    assert np.all(np.diff(nnz[work]) <= 0)
-    # ties keep unit order
-    for a, b in zip(work, work[1:]):
-        if nnz[a] == nnz[b]:
-            assert a < b
+    heads = work // 7
+    assert heads.tolist() == sorted(heads.tolist())  # head by head, in index order
+    for h in range(3):
+        w = work[heads == h]
+        assert np.all(np.diff(nnz[w]) <= 0)  # longest first inside a head
+        for a, b in zip(w, w[1:]):
+            if nnz[a] == nnz[b]:
+                assert a < b  # ties keep block order
     work = binding.build_plan(rp, 3, 7, head_active=np.array([0, 1, 0], np.uint8))
     assert sorted(work.tolist()) == list(range(7, 14))
 
@@ -150,6 +153,26 @@ def test_argument_errors_are_caught_on_the_host(binding):
     assert lib.calibatt_spatial_score(fake, 1, 2, 8, 16, 5, float("nan"), fake, None, None) == -1
     assert lib.calibatt_spatial_score(fake, 1, 2, 8, 16, 5, 0.87, None, None, None) == -1
     assert lib.calibatt_spatial_score(odd2, 1, 2, 8, 16, 5, 0.87, fake, None, None) == -3
+    # mixed launch: too many units, k above H, missing workspace
+    assert lib.calibatt_mixed_attn_fwd(fake, fake, fake, 2, 2, 8, 16, 128, 5, 0.1, fake, fake, 4, fake, 1, fake,
+                                       100, fake, None, fake, 1 << 30, None) == -1
+    assert lib.calibatt_mixed_attn_fwd(fake, fake, fake, 2, 2, 4, 16, 128, 5, 0.1, fake, fake, 4, fake, 1, fake,
+                                       2, fake, None, fake, 1 << 30, None) == -1
+    assert lib.calibatt_mixed_attn_fwd(fake, fake, fake, 2, 2, 8, 16, 128, 5, 0.1, fake, fake, 4, fake, 1, fake,
+                                       2, fake, None, None, 0, None) == -1
+
+
+def test_mixed_plan_orders_both_kinds_of_units(binding):
+    # 3 heads, nb = 4; head 1 repeated; F*k*W = 2*5*30 = 300 anchor queries -> 3 anchor blocks
+    heads, nb, F, H, W, kk = 3, 4, 2, 10, 30, 5
+    counts = np.array([[4, 0, 2, 1], [9, 9, 9, 9], [3, 4, 1, 4]], np.int32)
+    row_ptr = np.concatenate([[0], np.cumsum(counts.reshape(-1))]).astype(np.int32)
+    work = binding.build_mixed_plan(row_ptr, heads, nb, [1], F, H, W, kk)
+    # head 1's anchor units, then head 0 and head 2 longest first (ties in block order)
+    assert work.tolist() == [12, 13, 14, 0, 2, 3, 1, 9, 11, 8, 10]
+    # no repeated heads: the plain plan
+    plain = binding.build_mixed_plan(row_ptr, heads, nb, [], F, H, W, kk)
+    np.testing.assert_array_equal(plain, binding.build_plan(row_ptr, heads, nb))
 
 
 def test_workspace_sizes(binding):

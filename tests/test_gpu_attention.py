@@ -146,3 +146,69 @@ def test_malformed_skip_list_is_reported_not_faulted():
                             torch.from_numpy(bad).to(dev), torch.tensor([0, 1], dtype=torch.int32, device=dev))
     assert binding.get_status() == -2  # CALIBATT_ERR_CSR
     assert binding.get_status() == 0   # cleared
+
+
+@pytest.mark.parametrize("F,H,W,kk,keep,seed", [(3, 8, 16, 5, 0.4, 1), (2, 30, 5, 5, 0.5, 2), (4, 5, 9, 2, 0.3, 3),
+                                                (2, 45, 8, 5, 0.35, 4)])
+def test_mixed_launch_matches_oracle_and_separate_calls(oracle, F, H, W, kk, keep, seed):
+    """Block-sparse and repeated heads in one persistent launch: each head
+    against the oracle, and bit for bit the outputs of the two separate calls
+    (a unit's arithmetic does not depend on which slot runs it)."""
+    binding = require_gpu()
+    heads = 4
+    n = F * H * W
+    nb = (n + 127) // 128
+    q, k, v = synth.plain_qkv(heads, n, seed=40 + seed)
+    rng = np.random.default_rng(seed)
+    mask = (rng.random((heads, nb, nb)) < keep).astype(np.uint8)
+    mask[:, np.arange(nb), np.arange(nb)] = 1
+    rep = [1, 3]
+    sparse = [0, 2]
+    row_ptr, col_idx = oracle.mask_to_csr(mask)
+    work = binding.build_mixed_plan(row_ptr, heads, nb, rep, F, H, W, kk)
+    dev = torch.device("cuda")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    rp_d, ci_d = torch.from_numpy(row_ptr).to(dev), torch.from_numpy(col_idx).to(dev)
+    rep_d = torch.tensor(rep, dtype=torch.int32, device=dev)
+    o, lse = binding.mixed_attn_fwd(qd, kd, vd, F, H, W, rp_d, ci_d, rep_d, torch.from_numpy(work).to(dev),
+                                    k_anchor=kk)
+    assert binding.get_status() == 0
+    # against the oracle
+    og = bf16_to_f64(o)
+    o_ref, lse_ref = oracle.masked_attention(synth.bf16_bits(q[sparse]), synth.bf16_bits(k[sparse]),
+                                             synth.bf16_bits(v[sparse]), mask[sparse])
+    assert attn_tolerance_ok(og[sparse], o_ref)[0]
+    o_rep, lse_rep = oracle.repeat_attention(synth.bf16_bits(q[rep]), synth.bf16_bits(k[rep]),
+                                             synth.bf16_bits(v[rep]), F, H, W, k_anchor=kk)
+    assert attn_tolerance_ok(og[rep], o_rep)[0]
+    np.testing.assert_allclose(lse.cpu().numpy()[rep], lse_rep, rtol=0, atol=2e-3)
+    # against the two separate calls, bit for bit
+    ha = np.ones(heads, np.uint8)
+    ha[rep] = 0
+    work_s = torch.from_numpy(binding.build_plan(row_ptr, heads, nb, head_active=ha)).to(dev)
+    o2 = torch.zeros_like(qd)
+    lse2 = torch.zeros((heads, n), dtype=torch.float32, device=dev)
+    binding.sparse_attn_fwd(qd, kd, vd, rp_d, ci_d, work_s, o=o2, lse=lse2)
+    binding.repeat_attn_fwd(qd, kd, vd, F, H, W, rep_d, k_anchor=kk, o=o2, lse=lse2)
+    assert binding.get_status() == 0
+    assert torch.equal(o, o2)
+    assert torch.equal(lse, lse2)
+
+
+def test_mixed_launch_without_repeated_heads_is_the_sparse_call(oracle):
+    binding = require_gpu()
+    F, H, W, heads = 2, 8, 16, 2
+    n = F * H * W
+    nb = (n + 127) // 128
+    q, k, v = synth.plain_qkv(heads, n, seed=60)
+    mask = np.ones((heads, nb, nb), np.uint8)
+    mask[0, 0, 1] = 0
+    row_ptr, col_idx = oracle.mask_to_csr(mask)
+    dev = torch.device("cuda")
+    args = [t.to(dev) for t in (q, k, v)]
+    rp_d, ci_d = torch.from_numpy(row_ptr).to(dev), torch.from_numpy(col_idx).to(dev)
+    work = torch.from_numpy(binding.build_mixed_plan(row_ptr, heads, nb, [], F, H, W)).to(dev)
+    o, lse = binding.mixed_attn_fwd(*args, F, H, W, rp_d, ci_d, torch.zeros(0, dtype=torch.int32, device=dev), work)
+    o2, lse2 = binding.sparse_attn_fwd(*args, rp_d, ci_d, torch.from_numpy(binding.build_plan(row_ptr, heads, nb)).to(dev))
+    assert binding.get_status() == 0
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)

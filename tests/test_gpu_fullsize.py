@@ -211,3 +211,27 @@ def test_spatial_classification_full_size(oracle, name):
                                                   int(g % rows_per_head) for g in sample], np.int64),
                                   threads=min(16, os.cpu_count() or 1))
     assert _energy_ok(got.reshape(-1, got.shape[-1])[sample], ref)
+
+
+def test_wan720_mixed_launch_equals_separate_calls():
+    """The benchmark's step (one launch for the 32 block-sparse and 8 repeated
+    heads) gives bit for bit the outputs of the separate calls, whose rows the
+    test above checks against the oracle."""
+    binding = require_gpu()
+    wl = synth.WORKLOADS["wan720"]
+    dev = torch.device(DEV)
+    q, k, v = synth.qkv(wl, 8, device=dev)
+    masks = synth.random_block_masks(wl)
+    row_ptr, col_idx = _skiplist(binding, masks, dev)
+    rp_h = row_ptr.cpu().numpy()
+    rep = list(wl.repeat_heads)
+    rep_d = torch.tensor(rep, dtype=torch.int32, device=dev)
+    work = torch.from_numpy(binding.build_mixed_plan(rp_h, wl.heads, wl.nb, rep, wl.F, wl.H, wl.W)).to(dev)
+    o, lse = binding.mixed_attn_fwd(q, k, v, wl.F, wl.H, wl.W, row_ptr, col_idx, rep_d, work)
+    ha = np.array([h not in rep for h in range(wl.heads)], np.uint8)
+    work_s = torch.from_numpy(binding.build_plan(rp_h, wl.heads, wl.nb, ha)).to(dev)
+    o2, lse2 = binding.sparse_attn_fwd(q, k, v, row_ptr, col_idx, work_s)
+    binding.repeat_attn_fwd(q, k, v, wl.F, wl.H, wl.W, rep_d, o=o2, lse=lse2)
+    assert binding.get_status() == 0
+    assert torch.equal(o, o2)
+    assert torch.equal(lse, lse2)
