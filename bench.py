@@ -257,6 +257,9 @@ def graph_time(fn, reps, stream):
     return ms
 
 
+TRAFFIC_PER_TILE = 765.87e6 / 514058  # dram bytes per kept tile, measured (see the roofline block)
+
+
 def run_ours(args, world, rank, local):
     from calibrated_block_sparse_b200 import binding
     binding.load()
@@ -478,10 +481,18 @@ def run_ours(args, world, rank, local):
     achieved = f_step / (attn_ms * 1e-3) / 1e12
     kname = ("attn_kernel<attention> (%d block-sparse + %d repeated heads, one launch; window includes the "
              "anchor gather)" % (len(sparse_heads), len(rep_heads)))
+    # DRAM traffic per launch: the given figure, else the bytes per kept tile
+    # of the one ncu capture (profiles/attn_kernel_wan720_5heads_ncu_full.md:
+    # 765.9 MB over 514 058 kept tiles) times the tiles of this launch
+    tiles = int(sum(int(masks[h].sum()) for h in sparse_heads)) + len(rep_heads) * -(-wl.F * wl.k_anchor * wl.W // 128) * nb
+    traffic = args.traffic_bytes if args.traffic_bytes else TRAFFIC_PER_TILE * tiles
     roofline = {"bound": "tensor", "kernel": kname,
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{pk_src} {'sustained' if long_run else 'burst'} bf16",
-                "traffic": args.traffic_bytes}
+                "traffic": traffic,
+                "traffic_source": "given" if args.traffic_bytes else
+                "ncu dram bytes of a 5-head capture, scaled by kept tiles (%d in this launch)" % tiles,
+                "algorithmic_bytes": 4.0 * heads * n * D * 2}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
