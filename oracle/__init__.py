@@ -282,3 +282,17 @@ def spatial_score(Epx, F, H, k_anchor=5):
 def repeat_flag(s, gamma=0.87):
     """A head is spatially repeated when its score exceeds gamma (explainer §三)."""
     return bool(s > gamma)
+
+
+def keep_histogram(counts, n_inputs):
+    """Keep-rate histogram of calibrated blocks (explainer §二 observation 3:
+    over the calibration inputs a block is almost always kept or almost always
+    skipped, so the histogram of count / n is bimodal): for each head, the
+    number of blocks kept by exactly c of the n inputs, c = 0..n.
+
+    counts: [heads, ...] integer mask counts over n_inputs inputs.
+    Returns int64 [heads][n_inputs + 1]."""
+    c = np.asarray(counts).reshape(np.asarray(counts).shape[0], -1).astype(np.int64)
+    if c.size and (c.min() < 0 or c.max() > n_inputs):
+        raise ValueError("a count lies outside [0, n_inputs]")
+    return np.stack([np.bincount(row, minlength=n_inputs + 1) for row in c]).astype(np.int64)

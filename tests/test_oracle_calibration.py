@@ -205,3 +205,27 @@ def test_eps_schedule_closed_form(oracle):
     ts = [oracle.eps_schedule(A, C, 5, t, 50) for t in range(51)]
     assert all(a > b for a, b in zip(ts, ts[1:]))
     assert oracle.eps_schedule(A, C, 5, 1e9, 1.0) == A
+
+
+# ---------------------------------------------------------------- keep-rate histogram
+
+def test_keep_histogram_counts_every_block(oracle):
+    rng = np.random.default_rng(31)
+    masks = (rng.random((16, 3, 9, 9)) < 0.3).astype(np.uint8)
+    _, counts = oracle.aggregate(masks, 0.5)
+    hist = oracle.keep_histogram(counts, 16)
+    assert hist.shape == (3, 17)
+    np.testing.assert_array_equal(hist.sum(-1), 81)
+    # the histogram's first moment is the total number of kept (input, block) pairs
+    np.testing.assert_array_equal((hist * np.arange(17)).sum(-1), masks.sum(axis=(0, 2, 3)))
+
+
+def test_keep_histogram_small_cases(oracle):
+    # one input: the histogram is (#skipped, #kept) of the mask itself
+    mask = np.array([[[1, 0, 0], [1, 1, 0], [0, 0, 0]]], np.uint8)
+    np.testing.assert_array_equal(oracle.keep_histogram(mask, 1), [[6, 3]])
+    # hand-made counts over 4 inputs
+    counts = np.array([[[0, 4, 4], [2, 0, 4]]])
+    np.testing.assert_array_equal(oracle.keep_histogram(counts, 4), [[2, 0, 1, 0, 3]])
+    with pytest.raises(ValueError):
+        oracle.keep_histogram(np.array([[5]]), 4)
