@@ -70,6 +70,12 @@ def load(build_if_missing: bool = False):
             "calibatt_aggregate_masks_noalloc": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P]),
             "calibatt_pixel_row_energy": (i32, [P, P, i32, i32, i32, i32, i32, f32, P, P, P, P]),
             "calibatt_build_mixed_plan": (i32, [P, i32, i32, P, i32, P, i32, i32, i32, i32, P, P]),
+            "calibatt_keep_histogram": (i32, [P, i32, i64, i32, P, P]),
+            "calibatt_bank_create": (P, [i32, i32, i32, i32, i32, i32, i32]),
+            "calibatt_bank_destroy": (None, [P]),
+            "calibatt_bank_entry_bytes": (sz, [P, i64, i32]),
+            "calibatt_bank_put": (i32, [P, i32, i32, f64, P, P, i64, P, i32, P, sz, P]),
+            "calibatt_bank_get": (i32, [P, i32, i32, P]),
             "calibatt_mixed_attn_fwd": (i32, [P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, i64, P, i32, P, i32,
                                               P, P, P, sz, P]),
             "calibatt_spatial_score": (i32, [P, i32, i32, i32, i32, i32, f32, P, P, P]),
@@ -387,3 +393,90 @@ def aggregate_masks_noalloc(counts, n_inputs, rho, mask, row_ptr, col_idx, nnz, 
                                                  _stream(stream))
     _check(rc, "calibatt_aggregate_masks_noalloc")
     return mask, row_ptr, col_idx, nnz
+
+
+# ------------------------------------------------------------------ calibration bank
+
+def keep_histogram(counts, n_inputs, stream=None):
+    """Per head, the number of blocks kept by exactly c of the n_inputs inputs: int64 [heads][n_inputs + 1]."""
+    _cuda_tensor(counts, torch.uint16, "counts")
+    heads = counts.shape[0]
+    cells = counts.numel() // heads
+    hist = torch.empty((heads, n_inputs + 1), dtype=torch.int64, device=counts.device)
+    rc = load().calibatt_keep_histogram(_ptr(counts), heads, cells, int(n_inputs), _ptr(hist), _stream(stream))
+    _check(rc, "calibatt_keep_histogram")
+    return hist
+
+
+class BankEntry(ctypes.Structure):
+    _fields_ = [("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p), ("nnz", ctypes.c_int64),
+                ("work_list", ctypes.c_void_p), ("n_work", ctypes.c_int32), ("rep_heads", ctypes.c_void_p),
+                ("n_rep", ctypes.c_int32), ("eps", ctypes.c_double)]
+
+
+class MaskBank:
+    """The (t, l) mask bank (calibatt_bank_*): entry buffers are torch device
+    tensors this object keeps alive; lookups return views of them."""
+
+    def __init__(self, timesteps, layers, heads, F, H, W, k_anchor=5):
+        self._lib = load()
+        self._h = self._lib.calibatt_bank_create(timesteps, layers, heads, F, H, W, k_anchor)
+        if not self._h:
+            raise CalibattError(-1, "calibatt_bank_create: bad sizes")
+        self.shape = (timesteps, layers, heads, F, H, W, k_anchor)
+        self._buffers = {}
+
+    def close(self):
+        if self._h:
+            self._lib.calibatt_bank_destroy(self._h)
+            self._h = None
+        self._buffers.clear()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def put(self, t, l, eps, row_ptr, col_idx, rep_heads=(), stream=None):
+        """Store entry (t, l): row_ptr (device or host int32), col_idx (device int32), rep_heads (ints)."""
+        _cuda_tensor(col_idx, torch.int32, "col_idx")
+        rp = np.ascontiguousarray(row_ptr.cpu().numpy() if isinstance(row_ptr, torch.Tensor) else row_ptr, np.int32)
+        rep = np.ascontiguousarray([int(h) for h in rep_heads], np.int32)
+        nnz = col_idx.numel()
+        need = self._lib.calibatt_bank_entry_bytes(self._h, nnz, len(rep))
+        if need == 0:
+            raise CalibattError(-1, "calibatt_bank_entry_bytes")
+        buf = torch.empty(need + 256, dtype=torch.uint8, device=col_idx.device)
+        off = (-buf.data_ptr()) % 256
+        rc = self._lib.calibatt_bank_put(self._h, t, l, float(eps), _ptr(rp), _ptr(col_idx) if nnz else None, nnz,
+                                         _ptr(rep) if len(rep) else None, len(rep), buf.data_ptr() + off, need,
+                                         _stream(stream))
+        _check(rc, "calibatt_bank_put")
+        self._buffers[(t, l)] = (buf, off)
+
+    def get(self, t, l):
+        """Entry (t, l) as tensors viewing its buffer: dict of row_ptr, col_idx,
+        work_list, rep_heads (device int32) and eps."""
+        e = BankEntry()
+        _check(self._lib.calibatt_bank_get(self._h, t, l, ctypes.byref(e)), "calibatt_bank_get")
+        buf, _ = self._buffers[(t, l)]
+        base = buf.data_ptr()
+
+        def view(ptr, count):
+            if count == 0:
+                return torch.empty(0, dtype=torch.int32, device=buf.device)
+            start = ptr - base
+            return buf[start:start + 4 * count].view(torch.int32)
+
+        _, _, heads, F, H, W, _ = self.shape
+        nb = -(-F * H * W // BLOCK)
+        return {"row_ptr": view(e.row_ptr, heads * nb + 1), "col_idx": view(e.col_idx, e.nnz),
+                "work_list": view(e.work_list, e.n_work), "rep_heads": view(e.rep_heads, e.n_rep), "eps": e.eps}
+
+    def attention(self, q, k, v, t, l, o=None, lse=None, stream=None):
+        """Online inference for step t, layer l: one mixed launch over the entry's lists."""
+        _, _, _, F, H, W, k_anchor = self.shape
+        e = self.get(t, l)
+        return mixed_attn_fwd(q, k, v, F, H, W, e["row_ptr"], e["col_idx"], e["rep_heads"], e["work_list"],
+                              k_anchor=k_anchor, o=o, lse=lse, stream=stream)

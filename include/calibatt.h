@@ -267,6 +267,63 @@ int calibatt_pixel_row_energy(const calibatt_bf16* q, const calibatt_bf16* k, in
 int calibatt_spatial_score(const float* pix_energy, int heads, int frames, int H, int nb, int k_anchor,
                            float gamma, float* score, uint8_t* flag, calibatt_stream_t stream);
 
+/* ---------------------------------------------------------------- calibration bank */
+
+/* Keep-rate histogram of calibrated blocks (explainer §二 observation 3: over
+ * the calibration inputs most blocks are kept by almost all of them or by
+ * almost none, a bimodal histogram of count / n): for each head,
+ * hist[h][c] = number of blocks kept by exactly c of the n_inputs inputs.
+ *   counts : device uint16 [heads][cells] (calibatt_accumulate_masks or the
+ *            fused selection of calibatt_block_energy)
+ *   hist   : device int64 [heads][n_inputs + 1] (output; cleared first)
+ * Counts above n_inputs go to the last bin and are reported through
+ * calibatt_get_status as CALIBATT_ERR_ARG. Requires n_inputs <= 4096. */
+int calibatt_keep_histogram(const uint16_t* counts, int heads, int64_t cells, int n_inputs, int64_t* hist,
+                            calibatt_stream_t stream);
+
+/* The (t, l) mask bank read by online inference (explainer §三: calibration
+ * runs once offline; online, each step looks up the skip list or the repeat
+ * marks of its (t, l, h) with no decision at run time). A bank is a host-side
+ * index over device memory the caller owns: calibatt_bank_put copies one
+ * entry (skip list, work list, repeated heads) into a caller buffer of
+ * calibatt_bank_entry_bytes and records where it is; calibatt_bank_get hands
+ * the device pointers back for calibatt_mixed_attn_fwd. Keep each entry's
+ * buffer alive while the bank is used. */
+typedef struct calibatt_bank calibatt_bank;
+
+typedef struct calibatt_bank_entry {
+  const int32_t* row_ptr;   /* device int32 [heads*nb + 1] */
+  const int32_t* col_idx;   /* device int32 [nnz] */
+  int64_t nnz;
+  const int32_t* work_list; /* device int32 [n_work] (calibatt_build_mixed_plan order) */
+  int32_t n_work;
+  const int32_t* rep_heads; /* device int32 [n_rep] */
+  int32_t n_rep;
+  double eps;               /* energy threshold of the calibration, eps(t) */
+} calibatt_bank_entry;
+
+/* A bank of timesteps x layers entries for heads heads of frames x H x W
+ * tokens and k_anchor anchor rows; NULL on bad sizes or no host memory. */
+calibatt_bank* calibatt_bank_create(int timesteps, int layers, int heads, int frames, int H, int W, int k_anchor);
+void calibatt_bank_destroy(calibatt_bank* bank);
+
+/* Device bytes of one entry with nnz kept blocks and n_rep repeated heads
+ * (0 on bad arguments). */
+size_t calibatt_bank_entry_bytes(const calibatt_bank* bank, int64_t nnz, int n_rep);
+
+/* Stores entry (t, l), calibrated at eps, replacing any earlier one: copies
+ * row_ptr (host int32 [heads*nb + 1]), col_idx (device int32 [nnz]) and
+ * rep_heads (host int32 [n_rep]) into dst, with the work list that
+ * calibatt_build_mixed_plan makes of them, on `stream`.
+ *   dst: device buffer of at least calibatt_bank_entry_bytes, 256-byte aligned
+ * Returns CALIBATT_ERR_CSR if row_ptr does not run from 0 to nnz. */
+int calibatt_bank_put(calibatt_bank* bank, int t, int l, double eps, const int32_t* row_ptr_host,
+                      const int32_t* col_idx, int64_t nnz, const int32_t* rep_heads_host, int n_rep, void* dst,
+                      size_t dst_bytes, calibatt_stream_t stream);
+
+/* Entry (t, l) (host only; CALIBATT_ERR_ARG if it was never stored). */
+int calibatt_bank_get(const calibatt_bank* bank, int t, int l, calibatt_bank_entry* out);
+
 /* ---------------------------------------------------------------- no-allocation variant */
 
 /* Largest heads * nb accepted by calibatt_aggregate_masks_noalloc. */

@@ -175,6 +175,35 @@ def test_mixed_plan_orders_both_kinds_of_units(binding):
     np.testing.assert_array_equal(plain, binding.build_plan(row_ptr, heads, nb))
 
 
+def test_bank_index_on_the_host(binding):
+    lib = binding.load()
+    P = ctypes.c_void_p
+    assert not lib.calibatt_bank_create(0, 2, 4, 2, 8, 16, 5)
+    assert not lib.calibatt_bank_create(2, 2, 4, 2, 4, 16, 5)  # k above H
+    b = lib.calibatt_bank_create(3, 2, 2, 2, 8, 16, 5)  # n = 256: nb = 2
+    assert b
+    try:
+        # [row_ptr 5 ints | col_idx 3 | work 4 + 2 anchor units | rep 1], each on 256 B
+        assert lib.calibatt_bank_entry_bytes(b, 3, 1) == 256 * 4
+        assert lib.calibatt_bank_entry_bytes(b, 3, 5) == 0
+        e = binding.BankEntry()
+        assert lib.calibatt_bank_get(b, 0, 0, ctypes.byref(e)) == -1  # never stored
+        assert lib.calibatt_bank_get(b, 3, 0, ctypes.byref(e)) == -1  # out of range
+        fake = P(0x100000)
+        rp = np.array([0, 1, 2, 2, 3], np.int32)
+        put = lambda rp_, dst, nbytes, t=0: lib.calibatt_bank_put(b, t, 0, 0.9, binding._ptr(rp_), fake, 3, None, 0,
+                                                                  dst, nbytes, None)
+        assert put(np.array([0, 1, 2, 2, 4], np.int32), fake, 4096) == -2  # row_ptr does not end at nnz
+        assert put(rp, P(0x100010), 4096) == -3                            # dst not 256-byte aligned
+        assert put(rp, fake, 16) == -1                                     # dst too small
+        assert put(rp, fake, 4096, t=3) == -1                              # t out of range
+    finally:
+        lib.calibatt_bank_destroy(b)
+    # keep-rate histogram arguments
+    assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 0, P(0x100000), None) == -1
+    assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 8, P(0x100004), None) == -3
+
+
 def test_workspace_sizes(binding):
     lib = binding.load()
     assert binding.repeat_workspace_size(8, 21, 45, 80, 5) == 8 * 21 * 5 * 80 * 256
