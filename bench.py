@@ -411,6 +411,15 @@ def run_ours(args, world, rank, local):
 
         energy_call()
         e_ms = cuda_time(energy_call, 2, stream)
+        ews = torch.empty(binding.energy_workspace_size(ch, n), dtype=torch.uint8, device=dev)
+
+        def energy1_call():
+            binding.block_energy_1pass(qc, kc, eps=0.9, energy=energy, mask=cmask, counts=ccounts, ws=ews,
+                                       stream=stream)
+
+        energy1_call()
+        e1_ms = cuda_time(energy1_call, 2, stream)
+        del ews
         f_energy_alg = float(2 * D * n * n * ch)  # one S = Q K^T per input
         f_energy_issued = 2 * f_energy_alg        # two passes recompute S
 
@@ -462,6 +471,7 @@ def run_ours(args, world, rank, local):
             "shape": f"{ch} heads x N={n}",
             "energy_ms": e_ms, "energy_tflops_algorithmic": f_energy_alg / (e_ms * 1e-3) / 1e12,
             "energy_tflops_issued": f_energy_issued / (e_ms * 1e-3) / 1e12,
+            "energy_1pass_ms": e1_ms, "energy_1pass_tflops": f_energy_alg / (e1_ms * 1e-3) / 1e12,
             "select_ms": s_ms, "select_gbs": sel_bytes / (s_ms * 1e-3) / 1e9,
             "aggregate_ms": a_ms, "aggregate_gbs": agg_bytes / (a_ms * 1e-3) / 1e9,
             "eps": 0.9, "kept_fraction_at_eps": float(cmask.float().mean().item()),

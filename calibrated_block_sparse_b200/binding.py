@@ -71,6 +71,8 @@ def load(build_if_missing: bool = False):
             "calibatt_pixel_row_energy": (i32, [P, P, i32, i32, i32, i32, i32, f32, P, P, P, P]),
             "calibatt_build_mixed_plan": (i32, [P, i32, i32, P, i32, P, i32, i32, i32, i32, P, P]),
             "calibatt_keep_histogram": (i32, [P, i32, i64, i32, P, P]),
+            "calibatt_energy_workspace_size": (sz, [i32, i32]),
+            "calibatt_block_energy_1pass": (i32, [P, P, i32, i32, i32, f32, P, sz, P, i32, f64, P, P, P, P, i32, P]),
             "calibatt_bank_create": (P, [i32, i32, i32, i32, i32, i32, i32]),
             "calibatt_bank_destroy": (None, [P]),
             "calibatt_bank_entry_bytes": (sz, [P, i64, i32]),
@@ -327,6 +329,39 @@ def spatial_score(pix, F, H, k_anchor=5, gamma=0.87, score=None, flag=True, stre
                                        _stream(stream))
     _check(rc, "calibatt_spatial_score")
     return score, flag
+
+
+def energy_workspace_size(heads: int, n: int) -> int:
+    return load().calibatt_energy_workspace_size(heads, n)
+
+
+def block_energy_1pass(q, k, eps=None, energy=True, mask=None, kept=None, counts=None, pix=None, pix_W=None,
+                       ws=None, scale=None, stream=None):
+    """Block energy of one input in a single pass over the keys (with eps, the
+    fused greedy selection too; with pix_W, pixel-row profiles of pix_W
+    consecutive queries). Returns (energy or None, mask, kept, counts, pix)."""
+    heads, n = _bhnd(q)
+    nb = (n + BLOCK - 1) // BLOCK
+    dev = q.device
+    if ws is None:
+        ws = torch.empty(energy_workspace_size(heads, n), dtype=torch.uint8, device=dev)
+    e = None
+    if energy is True:
+        e = torch.empty((heads, nb, nb), dtype=torch.float32, device=dev)
+    elif isinstance(energy, torch.Tensor):
+        e = energy
+    fuse = eps is not None
+    if fuse and mask is None and kept is None and counts is None:
+        mask = torch.empty((heads, nb, nb), dtype=torch.uint8, device=dev)
+        kept = torch.empty((heads, nb), dtype=torch.int32, device=dev)
+    if pix_W is not None and pix is None:
+        pix = torch.empty((heads, n // pix_W, nb), dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = load().calibatt_block_energy_1pass(_ptr(q), _ptr(k), heads, n, HEAD_DIM, scale, _ptr(ws), ws.numel(),
+                                            _ptr(e), 1 if fuse else 0, float(eps) if fuse else 0.0, _ptr(mask),
+                                            _ptr(kept), _ptr(counts), _ptr(pix), int(pix_W or 0), _stream(stream))
+    _check(rc, "calibatt_block_energy_1pass")
+    return e, mask, kept, counts, pix
 
 
 def select_mask(energy, eps, mask=True, kept=True, counts=None, stream=None):

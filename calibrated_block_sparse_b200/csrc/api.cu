@@ -14,6 +14,7 @@
 
 #include "calibatt.h"
 #include "kernels.h"
+#include "sched.cuh"
 
 namespace calibatt {
 
@@ -368,6 +369,57 @@ int calibatt_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int he
   p.kept = fuse_select ? kept : nullptr;
   p.counts = fuse_select ? counts : nullptr;
   return launch_attention(2, q, n, heads, k, nullptr, n, heads, p, st);
+}
+
+size_t calibatt_energy_workspace_size(int heads, int n) {
+  if (heads < 1 || n < 1) return 0;
+  const int64_t nb = (static_cast<int64_t>(n) + 127) / 128;
+  const int64_t units = heads * nb;
+  if (units > INT_MAX / 2 || nb > CALIBATT_MAX_CALIB_NB) return 0;
+  const size_t bytes = static_cast<size_t>(2 * score_grid(static_cast<int>(units))) * nb * 128 * sizeof(float2);
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int n, int d,
+                                float scale, void* ws, size_t ws_bytes, float* energy, int fuse_select, double eps,
+                                uint8_t* mask, int32_t* kept, uint16_t* counts, float* pix_energy, int pix_W,
+                                calibatt_stream_t stream) {
+  int rc = check_qkv(q, k, nullptr, nullptr, heads, n, d);
+  if (rc != CALIBATT_OK) return rc;
+  const int nb = (n + 127) / 128;
+  if (nb > CALIBATT_MAX_CALIB_NB) return CALIBATT_ERR_UNSUPPORTED;
+  if (!scale_ok(scale) || !ws || std::isnan(eps)) return CALIBATT_ERR_ARG;
+  if (ws_bytes < calibatt_energy_workspace_size(heads, n)) return CALIBATT_ERR_ARG;
+  if (fuse_select && !mask && !kept && !counts) return CALIBATT_ERR_ARG;
+  if (pix_energy && (pix_W < 1 || n % pix_W != 0)) return CALIBATT_ERR_ARG;
+  if (!aligned16(ws) || (energy && !aligned4(energy)) || (kept && !aligned4(kept)) ||
+      (counts && (reinterpret_cast<uintptr_t>(counts) & 1u)) || (pix_energy && !aligned4(pix_energy)))
+    return CALIBATT_ERR_ALIGN;
+  KernelParams p = base_params();
+  if (!p.status) return CALIBATT_ERR_CUDA;
+  p.n_q = p.n_k = n;
+  p.nbq = p.nbk = nb;
+  p.heads_q = p.heads_kv = heads;
+  p.n_units = heads * nb;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_out = n;
+  p.energy_ws = static_cast<float2*>(ws);
+  p.energy = energy;
+  p.fuse_select = fuse_select ? 1 : 0;
+  p.eps_fx = eps_to_fixed(eps);
+  p.mask = fuse_select ? mask : nullptr;
+  p.kept = fuse_select ? kept : nullptr;
+  p.counts = fuse_select ? counts : nullptr;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (pix_energy) {
+    const size_t pix_bytes = static_cast<size_t>(heads) * (n / pix_W) * nb * sizeof(float);
+    if (cudaMemsetAsync(pix_energy, 0, pix_bytes, st) != cudaSuccess) return CALIBATT_ERR_CUDA;
+    p.pix_energy = pix_energy;
+    p.pix_W = pix_W;
+    p.pix_rows = n / pix_W;
+    p.pix_inv_W = 1.0f / static_cast<float>(pix_W);
+  }
+  return launch_attention(3, q, n, heads, k, nullptr, n, heads, p, st);
 }
 
 int calibatt_select_mask(const float* energy, int heads, int nb, double eps, uint8_t* mask, int32_t* kept,

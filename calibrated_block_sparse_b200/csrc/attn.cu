@@ -404,7 +404,8 @@ int launch_attention(int mode, const void* q, int q_rows, int q_heads, const voi
   switch (mode) {
     case kAttn: return launch_attn(mq, mqb, mk, mv, p, stream);
     case kLse:
-    case kEnergy: return launch_score(mode, mq, mk, p, stream);
+    case kEnergy:
+    case kEnergy1: return launch_score(mode, mq, mk, p, stream);
     default: return CALIBATT_ERR_ARG;
   }
 }

@@ -48,6 +48,8 @@ struct KernelParams {
   float* pix_energy;   // [heads_q][pix_rows][nbk] or NULL
   int pix_W, pix_rows;
   float pix_inv_W;
+  // single-pass energy: per slot, per key block, per row (tile sum, running max)
+  float2* energy_ws;   // [2 * grid][nbk][128]
   int* status;         // device status word
 };
 
@@ -63,6 +65,8 @@ struct RowAnchorTable {
 
 // qb: the packed anchor tensor of the second unit segment ([qb_heads][qb_rows][128])
 // or NULL.
+// Modes of launch_attention: 0 attention, 1 row LSE pass, 2 energy pass
+// after it, 3 single-pass energy.
 int launch_attention(int mode, const void* q, int q_rows, int q_heads, const void* k, const void* v, int kv_rows,
                      int kv_heads, const KernelParams& p, cudaStream_t stream, const void* qb = nullptr,
                      int qb_rows = 0, int qb_heads = 0);

@@ -18,7 +18,7 @@ constexpr int kTile = 32768;  // one 128 x 128 bf16 tile
 constexpr int kHalf = 16384;  // one 64-column half (one TMA box)
 constexpr float kLn2 = 0.6931471805599453f;
 
-enum Mode : int { kAttn = 0, kLse = 1, kEnergy = 2 };
+enum Mode : int { kAttn = 0, kLse = 1, kEnergy = 2, kEnergy1 = 3 };
 
 // ------------------------------------------------------------------ work units
 struct Unit {
@@ -196,7 +196,13 @@ inline int sm_count() {
   return n;
 }
 
-// Energy-pass launcher (score.cu).
+// Energy-pass launcher (score.cu) and the grid it uses for n_units work units
+// (one CTA of two slots per SM at most).
 int launch_score(int mode, const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams& p, cudaStream_t stream);
+inline int score_grid(int n_units) {
+  const int sms = sm_count();
+  const int grid = (n_units + 1) / 2;
+  return grid > sms ? sms : grid;
+}
 
 }  // namespace calibatt

@@ -1,9 +1,15 @@
-// The two passes of the block-energy calibration (explainer §三, offline
-// calibration steps 1-2) on the tensor core: S = Q K^T tile by tile over all
-// key blocks, never storing P.
-//   pass 1 (kLse):    per query row, log2 sum_j 2^(scale' S_ij)  -> lse_ws
-//   pass 2 (kEnergy): per tile, sum_ij 2^(scale' S_ij - lse_i) -> E[r][c], then
-//                     the greedy eps selection of the finished row (select.cuh)
+// The block-energy calibration (explainer §三, offline calibration steps
+// 1-2) on the tensor core: S = Q K^T tile by tile over all key blocks, never
+// storing P.
+//   kLse:     per query row, log2 sum_j 2^(scale' S_ij)  -> lse_ws
+//   kEnergy:  second pass: per tile, sum_ij 2^(scale' S_ij - lse_i) -> E[r][c],
+//             then the greedy eps selection of the finished row (select.cuh)
+//   kEnergy1: the same energies in one pass: each row keeps its exact
+//             running max m and sum l, and stores every tile's sum t relative
+//             to m (with m) in a workspace; when the row is done,
+//             t * 2^(m - lse) gives its share of E[r][c] exactly as the second
+//             pass would, and the row's tiles are reduced and selected as
+//             above. S is computed once instead of twice.
 //
 // CTA (320 threads, one per SM): two query-tile slots; warps 0-3 and 4-7 are
 // the slots' row warpgroups (thread = query row = TMEM lane), warp 8 loads Q
@@ -58,7 +64,7 @@ struct ScoreLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTile;
   static constexpr int kAuxOff = kRingOff + kScoreRing * kTile;
-  static constexpr int kAuxBytes = (MODE == kEnergy) ? 2 * kEnergyScratch : 0;
+  static constexpr int kAuxBytes = (MODE == kEnergy || MODE == kEnergy1) ? 2 * kEnergyScratch : 0;
   static constexpr int kBarOff = kAuxOff + kAuxBytes;
   static constexpr int kBytes = kBarOff + static_cast<int>(sizeof(ScoreBarriers));
   static constexpr int kDynSmem = kBytes + 1024;  // + alignment slack
@@ -210,6 +216,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     uint32_t n_sfull = 0;
     bool ok = true;  // warp-uniform
     float* part = reinterpret_cast<float*>(smem + L::kAuxOff + s * kEnergyScratch);
+    // pixel-row profiles of key block j from each row's normalised tile sum v:
+    // a segmented scan over the warp's rows (a pixel row is a run of
+    // consecutive lanes), then one atomic add per pixel row from the run's
+    // last lane. Warp-collective.
+    int pix_key = -1;
+    int pix_hq = 0;
+    auto pix_add = [&](float v, int j) {
+      const int key = pix_key;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float vu = __shfl_up_sync(0xffffffffu, v, o);
+        const int ku = __shfl_up_sync(0xffffffffu, key, o);
+        if (lane >= o && ku == key) v += vu;
+      }
+      const int kn = __shfl_down_sync(0xffffffffu, key, 1);
+      if (ok && key >= 0 && (lane == 31 || kn != key))
+        atomicAdd(p.pix_energy + (static_cast<int64_t>(pix_hq) * p.pix_rows + key) * p.nbk + j, v * p.pix_inv_W);
+    };
 
     for (int round = 0;; ++round) {
       Unit u;
@@ -219,6 +243,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       const bool row_valid = qrow < p.n_q;
       float lse2 = 0.f;
       if (MODE == kEnergy && row_valid) lse2 = p.lse_ws[static_cast<int64_t>(u.hq) * p.nbq * 128 + qrow];
+      if (p.pix_energy) {
+        pix_key = row_valid ? qrow / p.pix_W : -1;
+        pix_hq = u.hq;
+      }
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < u.nnz; ++j) {
         const int buf = n_sfull & 1;
@@ -239,7 +267,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
               if (c >= nvalid) sv[c] = -INFINITY;
           }
           float ref;  // subtracted before the exponential
-          if (MODE == kLse) {
+          if (MODE == kLse || MODE == kEnergy1) {
             const float mx = row_max128(sv) * p.scale_log2;
             const float m_new = fmaxf(m_run, mx);
             if (m_run != -INFINITY) l_run *= ex2_approx(m_run - m_new);
@@ -248,7 +276,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           } else {
             ref = lse2;
           }
-          if (MODE == kLse || row_valid) {
+          if (MODE != kEnergy || row_valid) {
             const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
             const float2 nr2 = make_float2(-ref, -ref);
             float2 a4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -265,24 +293,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             const float2 s01 = fadd2(a4[0], a4[1]), s23 = fadd2(a4[2], a4[3]);
             acc = (s01.x + s01.y) + (s23.x + s23.y);
           }
-          if (MODE == kLse) l_run += acc;
+          if (MODE != kEnergy) l_run += acc;
+          // single pass: keep the tile's sum relative to the running max
+          if (MODE == kEnergy1)
+            p.energy_ws[(static_cast<int64_t>(g) * p.nbk + j) * 128 + row] = make_float2(acc, m_run);
         }
-        if (MODE == kEnergy && p.pix_energy) {
-          // pixel-row profiles: a segmented scan over the warp's rows (a
-          // pixel row is a run of consecutive lanes), then one atomic add per
-          // pixel row from the run's last lane
-          const int key = row_valid ? qrow / p.pix_W : -1;
-          float v = acc;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const float vu = __shfl_up_sync(0xffffffffu, v, o);
-            const int ku = __shfl_up_sync(0xffffffffu, key, o);
-            if (lane >= o && ku == key) v += vu;
-          }
-          const int kn = __shfl_down_sync(0xffffffffu, key, 1);
-          if (ok && key >= 0 && (lane == 31 || kn != key))
-            atomicAdd(p.pix_energy + (static_cast<int64_t>(u.hq) * p.pix_rows + key) * p.nbk + j, v * p.pix_inv_W);
-        }
+        if (MODE == kEnergy && p.pix_energy) pix_add(acc, j);
         if (MODE == kEnergy) {
           // this warp's share of E[r][j]: sum over its 32 rows
 #pragma unroll
@@ -293,6 +309,39 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       if (MODE == kLse) {
         if (ok) p.lse_ws[static_cast<int64_t>(u.hq) * p.nbq * 128 + qrow] = m_run + log2f(l_run);
       } else {
+        if (MODE == kEnergy1) {
+          // every tile sum rescaled to the row's final log-sum-exp, then
+          // summed over the warp's 32 rows, eight key blocks at a time
+          const float lse_r = m_run + log2f(l_run);
+          const float2* wsr = p.energy_ws + static_cast<int64_t>(g) * p.nbk * 128 + row;
+          for (int c0 = 0; c0 < p.nbk; c0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float x = 0.f;
+              if (ok && row_valid && c0 + i < p.nbk) {
+                const float2 w = wsr[static_cast<int64_t>(c0 + i) * 128];
+                x = w.x * ex2_approx(w.y - lse_r);
+              }
+              v[i] = x;
+            }
+            if (p.pix_energy) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                if (c0 + i < p.nbk) pix_add(v[i], c0 + i);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+            }
+            if (lane == 0) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                if (c0 + i < p.nbk) part[wl * 1024 + c0 + i] = v[i];
+            }
+          }
+        }
         named_bar_sync(1 + s, 128);
         const int rows = min(128, p.n_q - u.r * 128);
         const float inv_rows = 1.f / static_cast<float>(rows);
@@ -337,10 +386,7 @@ int launch_mode(const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams
     configured = true;
   }
   if (p.n_units <= 0) return CALIBATT_OK;
-  int grid = (p.n_units + 1) / 2;
-  const int sms = sm_count();
-  if (grid > sms) grid = sms;
-  score_kernel<MODE><<<grid, kScoreThreads, L::kDynSmem, stream>>>(mq, mk, p);
+  score_kernel<MODE><<<score_grid(p.n_units), kScoreThreads, L::kDynSmem, stream>>>(mq, mk, p);
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
 }
 
@@ -348,7 +394,12 @@ int launch_mode(const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams
 
 int launch_score(int mode, const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams& p,
                  cudaStream_t stream) {
-  return mode == kLse ? launch_mode<kLse>(mq, mk, p, stream) : launch_mode<kEnergy>(mq, mk, p, stream);
+  switch (mode) {
+    case kLse: return launch_mode<kLse>(mq, mk, p, stream);
+    case kEnergy: return launch_mode<kEnergy>(mq, mk, p, stream);
+    case kEnergy1: return launch_mode<kEnergy1>(mq, mk, p, stream);
+    default: return CALIBATT_ERR_ARG;
+  }
 }
 
 }  // namespace calibatt

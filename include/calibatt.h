@@ -191,6 +191,27 @@ int calibatt_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int he
                           float* lse_ws, float* energy, int fuse_select, double eps, uint8_t* mask,
                           int32_t* kept, uint16_t* counts, calibatt_stream_t stream);
 
+/* Workspace bytes of calibatt_block_energy_1pass for heads x n tokens on the
+ * current device (it depends on the number of SMs; 0 on bad sizes). */
+size_t calibatt_energy_workspace_size(int heads, int n);
+
+/* calibatt_block_energy in one pass over the keys instead of two: each query
+ * row keeps its exact running max m and running sum, and stores every key
+ * block's sum of 2^(scale' s - m) with m in ws; once the row's log-sum-exp
+ * is known the stored sums are rescaled and reduced into the same energies
+ * (and fused selection) as calibatt_block_energy, which computes S twice.
+ * With pix_energy != NULL it also writes the profiles of
+ * calibatt_pixel_row_energy for pixel rows of pix_W consecutive queries
+ * (pix_energy: device fp32 [heads][n / pix_W][nb], cleared first; pix_W must
+ * divide n).
+ *   ws : device scratch of calibatt_energy_workspace_size(heads, n) bytes,
+ *        16-byte aligned (no lse_ws is needed)
+ * Other arguments and outputs as in calibatt_block_energy. */
+int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int n, int d,
+                                float scale, void* ws, size_t ws_bytes, float* energy, int fuse_select, double eps,
+                                uint8_t* mask, int32_t* kept, uint16_t* counts, float* pix_energy, int pix_W,
+                                calibatt_stream_t stream);
+
 /* Greedy eps selection (explainer §三, step 3) on rows of block energies:
  * order the row's blocks by energy descending (equal energies: lower column
  * first) and keep the shortest prefix whose running sum reaches eps. The sum

@@ -199,6 +199,11 @@ def test_bank_index_on_the_host(binding):
         assert put(rp, fake, 4096, t=3) == -1                              # t out of range
     finally:
         lib.calibatt_bank_destroy(b)
+    # single-pass energy: short workspace, pixel rows that do not divide n
+    assert lib.calibatt_block_energy_1pass(P(0x100000), P(0x100000), 1, 4096, 128, 0.1, P(0x100000), 16, None, 0,
+                                           0.0, None, None, None, None, 0, None) == -1
+    assert lib.calibatt_block_energy_1pass(P(0x100000), P(0x100000), 1, 4096, 128, 0.1, P(0x100000), 1 << 40,
+                                           None, 0, 0.0, None, None, None, P(0x100000), 100, None) == -1
     # keep-rate histogram arguments
     assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 0, P(0x100000), None) == -1
     assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 8, P(0x100004), None) == -3

@@ -203,3 +203,65 @@ def test_select_with_many_equal_energies_is_exact(oracle, nb):
         m_ref, kept_ref = oracle.select(E.astype(np.float64), eps)
         np.testing.assert_array_equal(mask.cpu().numpy(), m_ref)
         np.testing.assert_array_equal(kept.cpu().numpy(), kept_ref)
+
+
+
+# ---------------------------------------------------------------- single-pass energy
+
+@pytest.mark.parametrize("heads,n,std,seed", [(1, 2048, 1.0, 1), (2, 1000, 2.0, 2), (1, 300, 3.0, 3),
+                                              (3, 128 * 40 + 7, 1.5, 4)])
+def test_single_pass_energy_matches_oracle(oracle, heads, n, std, seed):
+    binding = require_gpu()
+    q, k, _ = synth.plain_qkv(heads, n, seed=seed, std=std)
+    dev = torch.device("cuda")
+    qd, kd = q.to(dev), k.to(dev)
+    E1, _, _, _, _ = binding.block_energy_1pass(qd, kd)
+    assert binding.get_status() == 0
+    E1 = E1.cpu().numpy().astype(np.float64)
+    E_ref = oracle.block_energy(synth.bf16_bits(q), synth.bf16_bits(k))
+    ok, worst = _energy_ok(E1, E_ref)
+    assert ok, worst
+    np.testing.assert_allclose(E1.sum(-1), 1.0, atol=1e-4)
+
+
+def test_single_pass_fused_selection_and_profiles(oracle):
+    binding = require_gpu()
+    wl = synth.WORKLOADS["tiny"]
+    q, k, _ = synth.qkv(wl, 3, with_v=False)
+    dev = torch.device("cuda")
+    eps = 0.9
+    E, mask, kept, _, pix = binding.block_energy_1pass(q.to(dev), k.to(dev), eps=eps, pix_W=wl.W)
+    assert binding.get_status() == 0
+    E = E.cpu().numpy().astype(np.float64)
+    mask = mask.cpu().numpy()
+    E_ref = oracle.block_energy(synth.bf16_bits(q), synth.bf16_bits(k))
+    assert _energy_ok(E, E_ref)[0]
+    # the fused selection equals the oracle's selection of the same fp32 energies
+    m_same, _, cut_same = oracle.select(E, eps, with_cut=True)
+    n_diff, n_tie, bad = compare_masks(mask, m_same, tie_affected(cut_same, eps, 1e-6))
+    assert bad == 0, (n_diff, n_tie)
+    np.testing.assert_array_equal(kept.cpu().numpy(), mask.reshape(-1, mask.shape[-1]).sum(-1).reshape(kept.shape))
+    # pixel-row profiles from the same pass
+    P_ref = oracle.pixel_row_energy(synth.bf16_bits(q), synth.bf16_bits(k), wl.F, wl.H, wl.W)
+    assert _energy_ok(pix.cpu().numpy().astype(np.float64), P_ref)[0]
+
+
+def test_single_pass_counts_equal_two_pass_counts_away_from_ties(oracle):
+    """Calibrating 4 inputs with either energy kernel gives the same counts,
+    except blocks whose selection is tie-affected at the energy error bound."""
+    binding = require_gpu()
+    wl = synth.WORKLOADS["tiny"]
+    dev = torch.device("cuda")
+    nb = wl.nb
+    c1 = torch.zeros((wl.heads, nb, nb), dtype=torch.uint16, device=dev)
+    c2 = torch.zeros_like(c1)
+    aff = np.zeros((wl.heads, nb), bool)
+    for p in range(4):
+        q, k, _ = synth.qkv(wl, 10 + p, with_v=False, device=dev)
+        E1, _, _, _, _ = binding.block_energy_1pass(q, k, eps=0.9, counts=c1)
+        binding.block_energy(q, k, eps=0.9, energy=False, counts=c2)
+        _, _, cut = oracle.select(E1.cpu().numpy().astype(np.float64), 0.9, with_cut=True)
+        aff |= tie_affected(cut, 0.9, 1e-4)
+    assert binding.get_status() == 0
+    d = (c1 != c2).cpu().numpy().any(-1)
+    assert not np.any(d & ~aff), int((d & ~aff).sum())
