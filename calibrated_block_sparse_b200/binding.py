@@ -72,6 +72,9 @@ def load(build_if_missing: bool = False):
             "calibatt_build_mixed_plan": (i32, [P, i32, i32, P, i32, P, i32, i32, i32, i32, P, P]),
             "calibatt_keep_histogram": (i32, [P, i32, i64, i32, P, P]),
             "calibatt_energy_workspace_size": (sz, [i32, i32]),
+            "calibatt_mixed_host_workspace_size": (sz, [i32, i32, i32, i32, i32, i32, i32]),
+            "calibatt_mixed_attn_fwd_host": (i32, [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, P, i64, P,
+                                                   i32, i32, P, P, P, P, P, P, sz, P]),
             "calibatt_block_energy_1pass": (i32, [P, P, i32, i32, i32, f32, P, sz, P, i32, f64, P, P, P, P, i32, P]),
             "calibatt_bank_create": (P, [i32, i32, i32, i32, i32, i32, i32]),
             "calibatt_bank_destroy": (None, [P]),
@@ -256,6 +259,33 @@ def mixed_attn_fwd(q, k, v, F, H, W, row_ptr, col_idx, rep_heads, work_list, k_a
                                         _stream(stream))
     _check(rc, "calibatt_mixed_attn_fwd")
     return o, lse
+
+
+def mixed_attn_fwd_host(q_host, k_host, v_host, o_host, F, H, W, row_ptr_host, row_ptr, col_idx, rep_heads,
+                        q_dev, k_dev, v_dev, o_dev, lse_host=None, lse_dev=None, ws=None, heads_per_chunk=2,
+                        k_anchor=5, scale=None, stream=None):
+    """calibatt_mixed_attn_fwd from host buffers, copies overlapped with compute
+    over chunks of heads; o_host (lse_host) hold the result when `stream` is done."""
+    for t, name in ((q_host, "q_host"), (k_host, "k_host"), (v_host, "v_host"), (o_host, "o_host")):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host bf16 tensor")
+    heads, n = _bhnd(q_dev)
+    rp = np.ascontiguousarray(row_ptr_host, np.int32)
+    rep = np.ascontiguousarray([int(h) for h in rep_heads], np.int32)
+    lib = load()
+    if ws is None:
+        ws = torch.empty(lib.calibatt_mixed_host_workspace_size(heads, F, H, W, k_anchor, len(rep), heads_per_chunk),
+                         dtype=torch.uint8, device=q_dev.device)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = lib.calibatt_mixed_attn_fwd_host(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), o_host.data_ptr(),
+                                          lse_host.data_ptr() if lse_host is not None else None, heads, F, H, W,
+                                          HEAD_DIM, k_anchor, scale, _ptr(rp), _ptr(row_ptr),
+                                          _ptr(col_idx) if col_idx.numel() else None, col_idx.numel(),
+                                          _ptr(rep) if len(rep) else None, len(rep), int(heads_per_chunk),
+                                          _ptr(q_dev), _ptr(k_dev), _ptr(v_dev), _ptr(o_dev), _ptr(lse_dev), _ptr(ws),
+                                          ws.numel(), _stream(stream))
+    _check(rc, "calibatt_mixed_attn_fwd_host")
+    return o_host, lse_host
 
 
 # ------------------------------------------------------------------ calibration

@@ -297,6 +297,145 @@ int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, cons
   return launch_attention(0, q, n, heads, k, v, n, heads, p, st, n_rep > 0 ? ws : nullptr, p.n_q_b, n_rep);
 }
 
+// ------------------------------------------------------------------ host buffers
+// Streams and events of the host-buffer pipeline, created once per device
+// (copies in and out overlap the caller's compute stream).
+namespace {
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  std::vector<cudaEvent_t> ev;  // [start, end, in_0, done_0, in_1, done_1, ...]
+};
+
+std::mutex g_pipe_mu[64];
+
+// Caller holds g_pipe_mu[dev] for as long as it uses the pipe.
+int host_pipe(int dev, int n_chunks, HostPipe** out) {
+  static HostPipe pipes[64];
+  HostPipe& hp = pipes[dev];
+  if (!hp.in && (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
+                 cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess))
+    return CALIBATT_ERR_CUDA;
+  while (static_cast<int>(hp.ev.size()) < 2 + 2 * n_chunks) {
+    cudaEvent_t e;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return CALIBATT_ERR_CUDA;
+    hp.ev.push_back(e);
+  }
+  *out = &hp;
+  return CALIBATT_OK;
+}
+
+int64_t anchor_blocks(int frames, int W, int k_anchor) {
+  return (static_cast<int64_t>(frames) * k_anchor * W + 127) / 128;
+}
+}  // namespace
+
+size_t calibatt_mixed_host_workspace_size(int heads, int frames, int H, int W, int k_anchor, int n_rep,
+                                          int heads_per_chunk) {
+  if (heads < 1 || frames < 1 || H < 1 || W < 1 || k_anchor < 1 || k_anchor > H || n_rep < 0 || n_rep > heads)
+    return 0;
+  const int hpc = heads_per_chunk > 0 ? std::min(heads_per_chunk, heads) : std::min(2, heads);
+  const int64_t n = static_cast<int64_t>(frames) * H * W;
+  const int64_t nb = (n + 127) / 128;
+  const size_t anchors = n_rep > 0 ? calibatt_repeat_workspace_size(std::min(hpc, n_rep), frames, H, W, k_anchor) : 0;
+  const size_t lists = static_cast<size_t>(heads * nb + n_rep * anchor_blocks(frames, W, k_anchor) + n_rep) * 4;
+  return ((anchors + 255) & ~static_cast<size_t>(255)) + ((lists + 255) & ~static_cast<size_t>(255));
+}
+
+int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf16* k_host,
+                                 const calibatt_bf16* v_host, calibatt_bf16* o_host, float* lse_host, int heads,
+                                 int frames, int H, int W, int d, int k_anchor, float scale,
+                                 const int32_t* row_ptr_host, const int32_t* row_ptr, const int32_t* col_idx,
+                                 int64_t nnz, const int32_t* rep_heads_host, int32_t n_rep, int heads_per_chunk,
+                                 calibatt_bf16* q_dev, calibatt_bf16* k_dev, calibatt_bf16* v_dev,
+                                 calibatt_bf16* o_dev, float* lse_dev, void* ws, size_t ws_bytes,
+                                 calibatt_stream_t stream) {
+  if (!q_host || !k_host || !v_host || !o_host || !row_ptr_host || (lse_host && !lse_dev) || frames < 1 || H < 1 ||
+      W < 1 || n_rep < 0 || n_rep > heads || (n_rep > 0 && !rep_heads_host) || !ws)
+    return CALIBATT_ERR_ARG;
+  const int64_t n64 = static_cast<int64_t>(frames) * H * W;
+  if (n64 > INT_MAX / 2) return CALIBATT_ERR_ARG;
+  const int n = static_cast<int>(n64);
+  int rc = check_qkv(q_dev, k_dev, v_dev, o_dev, heads, n, d);
+  if (rc != CALIBATT_OK) return rc;
+  if (k_anchor < 1 || k_anchor > H) return CALIBATT_ERR_ARG;
+  if (ws_bytes < calibatt_mixed_host_workspace_size(heads, frames, H, W, k_anchor, n_rep, heads_per_chunk))
+    return CALIBATT_ERR_ARG;
+  if (!aligned16(ws) || (lse_dev && !aligned4(lse_dev))) return CALIBATT_ERR_ALIGN;
+  const int nb = (n + 127) / 128;
+  const int hpc = heads_per_chunk > 0 ? std::min(heads_per_chunk, heads) : std::min(2, heads);
+  const int n_chunks = (heads + hpc - 1) / hpc;
+  const int64_t nbq_b = anchor_blocks(frames, W, k_anchor);
+  for (int i = 0; i < n_rep; ++i)
+    if (rep_heads_host[i] < 0 || rep_heads_host[i] >= heads) return CALIBATT_ERR_ARG;
+  // every chunk's work list and repeated heads, staged to the device in one
+  // copy before any launch (a later pageable copy could wait for the stream)
+  std::vector<int32_t> lists;
+  std::vector<int> work_off(n_chunks), n_work(n_chunks), rep_off(n_chunks), n_rep_c(n_chunks);
+  std::vector<int32_t> plan(static_cast<size_t>(heads * nb + n_rep * nbq_b));
+  std::vector<uint8_t> active(static_cast<size_t>(heads));
+  for (int c = 0; c < n_chunks; ++c) {
+    const int h0 = c * hpc, h1 = std::min(heads, h0 + hpc);
+    std::vector<int32_t> rep_c;
+    for (int h = 0; h < heads; ++h) active[h] = (h >= h0 && h < h1) ? 1 : 0;
+    for (int i = 0; i < n_rep; ++i)
+      if (rep_heads_host[i] >= h0 && rep_heads_host[i] < h1) rep_c.push_back(rep_heads_host[i]);
+    int32_t nw = 0;
+    rc = calibatt_build_mixed_plan(row_ptr_host, heads, nb, active.data(), static_cast<int>(rep_c.size()),
+                                   rep_c.empty() ? nullptr : rep_c.data(), frames, H, W, k_anchor, plan.data(), &nw);
+    if (rc != CALIBATT_OK) return rc;
+    work_off[c] = static_cast<int>(lists.size());
+    lists.insert(lists.end(), plan.begin(), plan.begin() + nw);
+    n_work[c] = nw;
+    rep_off[c] = static_cast<int>(lists.size());
+    lists.insert(lists.end(), rep_c.begin(), rep_c.end());
+    n_rep_c[c] = static_cast<int>(rep_c.size());
+  }
+  const size_t anchor_bytes =
+      n_rep > 0 ? calibatt_repeat_workspace_size(std::min(hpc, n_rep), frames, H, W, k_anchor) : 0;
+  uint8_t* ws8 = static_cast<uint8_t*>(ws);
+  int32_t* lists_dev = reinterpret_cast<int32_t*>(ws8 + ((anchor_bytes + 255) & ~static_cast<size_t>(255)));
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CALIBATT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pipe_mu[dev]);  // one caller of a device's pipe at a time
+  HostPipe* hp = nullptr;
+  rc = host_pipe(dev, n_chunks, &hp);
+  if (rc != CALIBATT_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t head_elems = static_cast<size_t>(n) * 128;
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  if (!lists.empty() &&
+      !ok(cudaMemcpyAsync(lists_dev, lists.data(), lists.size() * 4, cudaMemcpyHostToDevice, st)))
+    return CALIBATT_ERR_CUDA;
+  // the device buffers may still be in use by earlier work on the stream
+  if (!ok(cudaEventRecord(hp->ev[0], st)) || !ok(cudaStreamWaitEvent(hp->in, hp->ev[0], 0)))
+    return CALIBATT_ERR_CUDA;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int h0 = c * hpc, h1 = std::min(heads, h0 + hpc);
+    const size_t off = static_cast<size_t>(h0) * head_elems, cnt = static_cast<size_t>(h1 - h0) * head_elems * 2;
+    cudaEvent_t ev_in = hp->ev[2 + 2 * c], ev_done = hp->ev[3 + 2 * c];
+    if (!ok(cudaMemcpyAsync(q_dev + off, q_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
+        !ok(cudaMemcpyAsync(k_dev + off, k_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
+        !ok(cudaMemcpyAsync(v_dev + off, v_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
+        !ok(cudaEventRecord(ev_in, hp->in)) || !ok(cudaStreamWaitEvent(st, ev_in, 0)))
+      return CALIBATT_ERR_CUDA;
+    rc = calibatt_mixed_attn_fwd(q_dev, k_dev, v_dev, heads, frames, H, W, d, k_anchor, scale, row_ptr, col_idx,
+                                 nnz, n_rep_c[c] ? lists_dev + rep_off[c] : nullptr, n_rep_c[c],
+                                 n_work[c] ? lists_dev + work_off[c] : nullptr, n_work[c], o_dev, lse_dev, ws,
+                                 anchor_bytes, stream);
+    if (rc != CALIBATT_OK) return rc;
+    if (!ok(cudaEventRecord(ev_done, st)) || !ok(cudaStreamWaitEvent(hp->out, ev_done, 0)) ||
+        !ok(cudaMemcpyAsync(o_host + off, o_dev + off, cnt, cudaMemcpyDeviceToHost, hp->out)) ||
+        (lse_host && !ok(cudaMemcpyAsync(lse_host + static_cast<size_t>(h0) * n, lse_dev + static_cast<size_t>(h0) * n,
+                                         static_cast<size_t>(h1 - h0) * n * sizeof(float), cudaMemcpyDeviceToHost,
+                                         hp->out))))
+      return CALIBATT_ERR_CUDA;
+  }
+  // the call is complete when the caller's stream is
+  if (!ok(cudaEventRecord(hp->ev[1], hp->out)) || !ok(cudaStreamWaitEvent(st, hp->ev[1], 0)))
+    return CALIBATT_ERR_CUDA;
+  return CALIBATT_OK;
+}
+
 size_t calibatt_repeat_workspace_size(int n_rep, int frames, int H, int W, int k_anchor) {
   if (n_rep < 1 || frames < 1 || H < 1 || W < 1 || k_anchor < 1) return 0;
   const size_t bytes = static_cast<size_t>(n_rep) * frames * k_anchor * W * 128 * 2;

@@ -170,6 +170,37 @@ int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, cons
                             const int32_t* work_list, int32_t n_work, calibatt_bf16* o, float* lse, void* ws,
                             size_t ws_bytes, calibatt_stream_t stream);
 
+/* Device workspace bytes of calibatt_mixed_attn_fwd_host (anchor queries of
+ * one chunk plus every chunk's work list); heads_per_chunk <= 0 means 2. */
+size_t calibatt_mixed_host_workspace_size(int heads, int frames, int H, int W, int k_anchor, int n_rep,
+                                          int heads_per_chunk);
+
+/* calibatt_mixed_attn_fwd on host buffers, pipelined over chunks of
+ * heads_per_chunk heads (<= 0: 2; on the Wan-720p workload 2 heads per chunk
+ * measured best of 2, 3, 4, 5, 8 and 20): while the attention of chunk c runs on
+ * `stream`, q, k, v of chunk c+1 are copied in on a second stream and o (and
+ * lse) of chunk c-1 copied out on a third, so copies and compute overlap.
+ * Returns once everything is enqueued; the results are in o_host (lse_host)
+ * when `stream` completes. Use page-locked host memory, else the copies do not
+ * overlap. The skip list, work lists and repeated heads are those of
+ * calibatt_mixed_attn_fwd; the work list of each chunk is built here from
+ * row_ptr_host.
+ *   q_host, k_host, v_host : host bf16 [heads][n][128]; o_host: host bf16 (output)
+ *   lse_host  : host fp32 [heads][n] or NULL (then lse_dev may be NULL)
+ *   row_ptr_host : host int32 [heads*nb + 1]; row_ptr, col_idx: the same list on the device
+ *   rep_heads_host : host int32 [n_rep]
+ *   q_dev, k_dev, v_dev, o_dev, lse_dev : device buffers of the full tensors
+ *   ws : device scratch of calibatt_mixed_host_workspace_size bytes
+ * Calls for one device are serialised on a host lock while they enqueue. */
+int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf16* k_host,
+                                 const calibatt_bf16* v_host, calibatt_bf16* o_host, float* lse_host, int heads,
+                                 int frames, int H, int W, int d, int k_anchor, float scale,
+                                 const int32_t* row_ptr_host, const int32_t* row_ptr, const int32_t* col_idx,
+                                 int64_t nnz, const int32_t* rep_heads_host, int32_t n_rep, int heads_per_chunk,
+                                 calibatt_bf16* q_dev, calibatt_bf16* k_dev, calibatt_bf16* v_dev,
+                                 calibatt_bf16* o_dev, float* lse_dev, void* ws, size_t ws_bytes,
+                                 calibatt_stream_t stream);
+
 /* ---------------------------------------------------------------- calibration */
 
 /* Block energy of one calibration input (explainer §三 offline calibration,

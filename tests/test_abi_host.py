@@ -204,6 +204,11 @@ def test_bank_index_on_the_host(binding):
                                            0.0, None, None, None, None, 0, None) == -1
     assert lib.calibatt_block_energy_1pass(P(0x100000), P(0x100000), 1, 4096, 128, 0.1, P(0x100000), 1 << 40,
                                            None, 0, 0.0, None, None, None, P(0x100000), 100, None) == -1
+    # host-buffer pipeline: short workspace, missing host buffer
+    assert lib.calibatt_mixed_attn_fwd_host(fake, fake, fake, fake, None, 2, 2, 8, 16, 128, 5, 0.1, fake, fake, fake,
+                                            4, None, 0, 8, fake, fake, fake, fake, None, fake, 4, None) == -1
+    assert lib.calibatt_mixed_attn_fwd_host(None, fake, fake, fake, None, 2, 2, 8, 16, 128, 5, 0.1, fake, fake, fake,
+                                            4, None, 0, 8, fake, fake, fake, fake, None, fake, 1 << 30, None) == -1
     # keep-rate histogram arguments
     assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 0, P(0x100000), None) == -1
     assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 8, P(0x100004), None) == -3

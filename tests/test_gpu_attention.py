@@ -212,3 +212,37 @@ def test_mixed_launch_without_repeated_heads_is_the_sparse_call(oracle):
     o2, lse2 = binding.sparse_attn_fwd(*args, rp_d, ci_d, torch.from_numpy(binding.build_plan(row_ptr, heads, nb)).to(dev))
     assert binding.get_status() == 0
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
+
+
+
+@pytest.mark.parametrize("chunk", [1, 2, 8])
+def test_host_buffer_pipeline_equals_device_call(oracle, chunk):
+    """calibatt_mixed_attn_fwd_host (copies in, compute, copies out, pipelined
+    over chunks of heads) returns bit for bit the device call's o and lse."""
+    binding = require_gpu()
+    F, H, W, heads, kk = 3, 8, 16, 5, 5
+    n = F * H * W
+    nb = (n + 127) // 128
+    q, k, v = synth.plain_qkv(heads, n, seed=70 + chunk)
+    rng = np.random.default_rng(chunk)
+    mask = (rng.random((heads, nb, nb)) < 0.5).astype(np.uint8)
+    mask[:, np.arange(nb), np.arange(nb)] = 1
+    rep = [1, 4]
+    row_ptr, col_idx = oracle.mask_to_csr(mask)
+    dev = torch.device("cuda")
+    rp_d, ci_d = torch.from_numpy(row_ptr).to(dev), torch.from_numpy(col_idx).to(dev)
+    rep_d = torch.tensor(rep, dtype=torch.int32, device=dev)
+    work = torch.from_numpy(binding.build_mixed_plan(row_ptr, heads, nb, rep, F, H, W, kk)).to(dev)
+    o_ref, lse_ref = binding.mixed_attn_fwd(q.to(dev), k.to(dev), v.to(dev), F, H, W, rp_d, ci_d, rep_d, work,
+                                            k_anchor=kk)
+    qh, kh, vh = (t.contiguous().pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(q).pin_memory()
+    lh = torch.empty((heads, n), dtype=torch.float32).pin_memory()
+    qd, kd, vd, od = (torch.empty_like(q, device=dev) for _ in range(4))
+    ld = torch.empty((heads, n), dtype=torch.float32, device=dev)
+    binding.mixed_attn_fwd_host(qh, kh, vh, oh, F, H, W, row_ptr, rp_d, ci_d, rep, qd, kd, vd, od, lse_host=lh,
+                                lse_dev=ld, heads_per_chunk=chunk, k_anchor=kk)
+    torch.cuda.synchronize()
+    assert binding.get_status() == 0
+    assert torch.equal(oh, o_ref.cpu())
+    assert torch.equal(lh, lse_ref.cpu())
