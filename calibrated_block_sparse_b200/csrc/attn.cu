@@ -277,10 +277,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (c >= valid_last) sv[c] = -INFINITY;
         }
-        float mx = sv[0];
-#pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
-        mx *= p.scale_log2;
+        const float mx = row_max128(sv) * p.scale_log2;  // eight independent 3-input max chains
         const float m_new = fmaxf(m_run, mx);
         // keep a stale running max unless it grew by more than the threshold
         // (P <= 2^8 stays exact enough in bf16/fp32 and O needs no rescale)
@@ -288,20 +285,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float m_use = need ? m_new : m_run;
         if (m_use == -INFINITY) m_use = 0.f;
         const float alpha = need ? ex2_approx(m_run - m_use) : 1.f;
-        float rs = 0.f;
+        // two keys at a time: packed fp32x2 multiply-add for s * scale' - m and
+        // packed adds into four partial row sums (half the issue slots of the
+        // scalar forms; measured 3 % faster on the full Wan-720p step)
+        float2 a4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 c2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-m_use, -m_use);
         uint32_t pk[32];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2_approx(fmaf(sv[h * 64 + 2 * i], p.scale_log2, -m_use));
-            const float p1 = ex2_approx(fmaf(sv[h * 64 + 2 * i + 1], p.scale_log2, -m_use));
-            rs += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            const float2 e = exp2_mufu2(ffma2(make_float2(sv[h * 64 + 2 * i], sv[h * 64 + 2 * i + 1]), c2, nm2));
+            a4[i & 3] = fadd2(a4[i & 3], e);
+            pk[i] = pack_bf16x2(e.x, e.y);
           }
           // P (bf16, two keys per column) over the first 64 columns of S
           tmem_st32(tmem + lane_off + s * 128 + h * 32, pk);
         }
+        const float2 s01 = fadd2(a4[0], a4[1]), s23 = fadd2(a4[2], a4[3]);
+        const float rs = (s01.x + s01.y) + (s23.x + s23.y);
         l_run = l_run * alpha + rs;
         m_run = m_use;
         // rescale the running O (its P V of block j-1 is complete: the
