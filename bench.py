@@ -257,7 +257,7 @@ def graph_time(fn, reps, stream):
     return ms
 
 
-TRAFFIC_PER_TILE = 765.87e6 / 514058  # dram bytes per kept tile, measured (see the roofline block)
+TRAFFIC_PER_TILE = 673.66e6 / 514058  # dram bytes per kept tile, measured (see the roofline block)
 
 
 def run_ours(args, world, rank, local):
@@ -496,7 +496,7 @@ def run_ours(args, world, rank, local):
              "anchor gather)" % (len(sparse_heads), len(rep_heads)))
     # DRAM traffic per launch: the given figure, else the bytes per kept tile
     # of the one ncu capture (profiles/attn_kernel_wan720_5heads_ncu_full.md:
-    # 765.9 MB over 514 058 kept tiles) times the tiles of this launch
+    # 673.7 MB over 514 058 kept tiles) times the tiles of this launch
     tiles = int(sum(int(masks[h].sum()) for h in sparse_heads)) + len(rep_heads) * -(-wl.F * wl.k_anchor * wl.W // 128) * nb
     traffic = args.traffic_bytes if args.traffic_bytes else TRAFFIC_PER_TILE * tiles
     roofline = {"bound": "tensor", "kernel": kname,
