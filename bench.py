@@ -184,6 +184,16 @@ def cpu_oracle_sample(wl, q_cpu, k_cpu, v_cpu, heads, masks, budget_s, rng, repe
     return spent, flops, rows_done, threads
 
 
+def arm_config(wl, heads, kept_frac, world):
+    """The workload description both arms print."""
+    sparse = [h for h in range(heads) if h not in wl.repeat_heads]
+    return {"workload": f"{wl.name}: {heads} heads x N={wl.n} (F={wl.F},H={wl.H},W={wl.W}), d={D}, "
+                        f"{len(sparse)} block-sparse + {heads - len(sparse)} repeated (k={wl.k_anchor})",
+            "kept_block_fraction": kept_frac, "block_sparsity": 1 - kept_frac,
+            "l2": "inputs (3 x %.2f GB) larger than L2; no flush" % (heads * wl.n * D * 2 / 1e9),
+            "parallelism": f"replica per GPU x{world}"}
+
+
 def run_reference(args, world, rank):
     """Reference arm: the oracle as it stands, on the host cores, same metric."""
     if rank != 0:
@@ -212,7 +222,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "heads": wl.heads, "n": wl.n, "d": D},
+        "config": arm_config(wl, wl.heads, float(np.mean([masks[h].mean() for h in sparse_heads])), world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -522,11 +532,7 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: {heads} heads x N={n} (F={wl.F},H={wl.H},W={wl.W}), d={D}, "
-                                   f"{len(sparse_heads)} block-sparse + {len(rep_heads)} repeated (k={wl.k_anchor})",
-                       "kept_block_fraction": kept_frac, "block_sparsity": 1 - kept_frac,
-                       "l2": "inputs (3 x %.2f GB) larger than L2; no flush" % (q.numel() * 2 / 1e9),
-                       "parallelism": f"replica per GPU x{world}"},
+            "config": arm_config(wl, heads, kept_frac, world),
             "gpu_launches": launches_per_step * args.steps,
             "attn_ms": attn_ms,
             "separate_calls": {"sparse_ms": sparse_ms, "repeat_ms": repeat_ms,
