@@ -184,14 +184,14 @@ def cpu_oracle_sample(wl, q_cpu, k_cpu, v_cpu, heads, masks, budget_s, rng, repe
     return spent, flops, rows_done, threads
 
 
-def arm_config(wl, heads, kept_frac, world):
+def arm_config(wl, heads, kept_frac, world, shard=False):
     """The workload description both arms print."""
     sparse = [h for h in range(heads) if h not in wl.repeat_heads]
     return {"workload": f"{wl.name}: {heads} heads x N={wl.n} (F={wl.F},H={wl.H},W={wl.W}), d={D}, "
                         f"{len(sparse)} block-sparse + {heads - len(sparse)} repeated (k={wl.k_anchor})",
             "kept_block_fraction": kept_frac, "block_sparsity": 1 - kept_frac,
             "l2": "inputs (3 x %.2f GB) larger than L2; no flush" % (heads * wl.n * D * 2 / 1e9),
-            "parallelism": f"replica per GPU x{world}"}
+            "parallelism": f"heads sharded over {world} GPUs" if shard else f"replica per GPU x{world}"}
 
 
 def run_reference(args, world, rank):
@@ -326,15 +326,25 @@ def run_ours(args, world, rank, local):
                                     stream=stream)
 
     # the step: block-sparse and repeated heads in one persistent launch
-    # (after the anchor gather), longest units first over both kinds
-    work_mixed = torch.from_numpy(binding.build_mixed_plan(row_ptr_h, heads, nb, rep_heads, wl.F, wl.H, wl.W,
-                                                           wl.k_anchor)).to(dev)
+    # (after the anchor gather). --shard heads: one call split over the ranks
+    # by heads (balanced by kept tiles, no exchange), strong scaling
+    shard = args.shard == "heads" and world > 1
+    if shard:
+        owner, _ = binding.shard_heads(row_ptr_h, heads, nb, rep_heads, wl.F, wl.W, wl.k_anchor, world)
+        work_np, my_rep = binding.build_rank_plan(row_ptr_h, heads, nb, rep_heads, owner, rank, wl.F, wl.H, wl.W,
+                                                  wl.k_anchor)
+        f_rank = sparse_flops(masks, [h for h in sparse_heads if owner[h] == rank], n) + repeat_flops(wl, len(my_rep))
+    else:
+        work_np = binding.build_mixed_plan(row_ptr_h, heads, nb, rep_heads, wl.F, wl.H, wl.W, wl.k_anchor)
+        my_rep, f_rank = rep_heads, f_step
+    work_mixed = torch.from_numpy(work_np).to(dev)
+    my_rep_t = torch.tensor(my_rep, dtype=torch.int32, device=dev)
 
     def step():
-        binding.mixed_attn_fwd(q, k, v, wl.F, wl.H, wl.W, row_ptr, col_idx, rep_t, work_mixed, wl.k_anchor, o=o,
+        binding.mixed_attn_fwd(q, k, v, wl.F, wl.H, wl.W, row_ptr, col_idx, my_rep_t, work_mixed, wl.k_anchor, o=o,
                                lse=lse, ws=ws, stream=stream)
 
-    launches_per_step = 1 + (1 if rep_heads else 0)
+    launches_per_step = 1 + (1 if my_rep else 0)
     for _ in range(args.warmup):
         step()
     binding.check_status(what="warmup")
@@ -361,10 +371,14 @@ def run_ours(args, world, rank, local):
     ms_step = elapsed_ms / args.steps
 
     # the same work as two separate calls (block-sparse, then repeated heads)
-    sparse_ms = cuda_time(sparse_call, max(2, min(5, args.steps)), stream)
-    repeat_ms = cuda_time(repeat_call, max(2, min(5, args.steps)), stream) if rep_heads else 0.0
-    binding.check_status(what="separate calls")
-    value = world * f_step / (ms_step * 1e-3) / 1e12
+    sparse_ms = repeat_ms = None
+    if not shard:
+        sparse_ms = cuda_time(sparse_call, max(2, min(5, args.steps)), stream)
+        repeat_ms = cuda_time(repeat_call, max(2, min(5, args.steps)), stream) if rep_heads else 0.0
+        binding.check_status(what="separate calls")
+    # weak scaling: every rank runs the whole call (replicas); strong: the
+    # ranks share one call
+    value = (1 if shard else world) * f_step / (ms_step * 1e-3) / 1e12
 
     # ---- 0 %-sparse run: the same kernel with every block kept, all 40 heads
     full = torch.ones((heads, nb, nb), dtype=torch.int16, device=dev).view(torch.uint16)
@@ -382,7 +396,7 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through the C ABI with host buffers: H2D q,k,v, call, D2H o
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not shard:
         qh = q.cpu().pin_memory()
         kh = k.cpu().pin_memory()
         vh = v.cpu().pin_memory()
@@ -501,13 +515,16 @@ def run_ours(args, world, rank, local):
     pk, pk_src = peaks()
     long_run = elapsed_ms > 1000.0
     peak = pk.get("bf16_tflops_sustained" if long_run else "bf16_tflops")
-    achieved = f_step / (attn_ms * 1e-3) / 1e12
+    achieved = f_rank / (attn_ms * 1e-3) / 1e12
     kname = ("attn_kernel<attention> (%d block-sparse + %d repeated heads, one launch; window includes the "
              "anchor gather)" % (len(sparse_heads), len(rep_heads)))
+    if shard:
+        kname += "; rank 0 share of the heads"
     # DRAM traffic per launch: the given figure, else the bytes per kept tile
     # of the one ncu capture (profiles/attn_kernel_wan720_5heads_ncu_full.md:
     # 673.7 MB over 514 058 kept tiles) times the tiles of this launch
-    tiles = int(sum(int(masks[h].sum()) for h in sparse_heads)) + len(rep_heads) * -(-wl.F * wl.k_anchor * wl.W // 128) * nb
+    mine = [h for h in sparse_heads if not shard or owner[h] == rank]
+    tiles = int(sum(int(masks[h].sum()) for h in mine)) + len(my_rep) * -(-wl.F * wl.k_anchor * wl.W // 128) * nb
     traffic = args.traffic_bytes if args.traffic_bytes else TRAFFIC_PER_TILE * tiles
     roofline = {"bound": "tensor", "kernel": kname,
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
@@ -530,13 +547,14 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if shard else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": arm_config(wl, heads, kept_frac, world),
+            "config": arm_config(wl, heads, kept_frac, world, shard),
             "gpu_launches": launches_per_step * args.steps,
             "attn_ms": attn_ms,
-            "separate_calls": {"sparse_ms": sparse_ms, "repeat_ms": repeat_ms,
-                               "sparse_tflops": f_sparse / (sparse_ms * 1e-3) / 1e12},
+            "separate_calls": None if shard else {"sparse_ms": sparse_ms, "repeat_ms": repeat_ms,
+                                                  "sparse_tflops": f_sparse / (sparse_ms * 1e-3) / 1e12},
             "dense_ms": dense_ms, "dense_tflops": f_dense / (dense_ms * 1e-3) / 1e12,
             "speedup_vs_dense": dense_ms / ms_step,
             "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "calibration": calib,
@@ -556,6 +574,8 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="run only the first HEADS heads (profiling case)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-chunk", type=int, default=2, help="heads per chunk of the host-buffer pipeline")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N>1: a replica of the call per rank (weak scaling) or one call split by heads (strong)")
     ap.add_argument("--no-calib", action="store_true")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="dram bytes per launch of the sparse kernel from an ncu capture")

@@ -72,6 +72,7 @@ def load(build_if_missing: bool = False):
             "calibatt_build_mixed_plan": (i32, [P, i32, i32, P, i32, P, i32, i32, i32, i32, P, P]),
             "calibatt_keep_histogram": (i32, [P, i32, i64, i32, P, P]),
             "calibatt_energy_workspace_size": (sz, [i32, i32]),
+            "calibatt_shard_heads": (i32, [P, i32, i32, P, i32, i32, i32, i32, i32, P, P]),
             "calibatt_mixed_host_workspace_size": (sz, [i32, i32, i32, i32, i32, i32, i32]),
             "calibatt_mixed_attn_fwd_host": (i32, [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, P, i64, P,
                                                    i32, i32, P, P, P, P, P, P, sz, P]),
@@ -170,6 +171,31 @@ def build_mixed_plan(row_ptr: np.ndarray, heads: int, nb: int, rep_heads, F: int
     _check(load().calibatt_build_mixed_plan(_ptr(rp), heads, nb, None, len(rep), _ptr(rep) if len(rep) else None,
                                             F, H, W, k_anchor, _ptr(out), _ptr(n)), "build_mixed_plan")
     return out[: int(n[0])].copy()
+
+
+def shard_heads(row_ptr: np.ndarray, heads: int, nb: int, rep_heads, F: int, W: int, k_anchor: int, n_ranks: int):
+    """Owner rank of every head and kept tiles per rank (calibatt_shard_heads)."""
+    rp = np.ascontiguousarray(row_ptr, np.int32)
+    rep = np.ascontiguousarray([int(h) for h in rep_heads], np.int32)
+    owner = np.empty(heads, np.int32)
+    load_ = np.empty(n_ranks, np.int64)
+    _check(load().calibatt_shard_heads(_ptr(rp), heads, nb, _ptr(rep) if len(rep) else None, len(rep), F, W, k_anchor,
+                                       n_ranks, _ptr(owner), _ptr(load_)), "shard_heads")
+    return owner, load_
+
+
+def build_rank_plan(row_ptr: np.ndarray, heads: int, nb: int, rep_heads, owner, rank: int, F: int, H: int, W: int,
+                    k_anchor: int = 5):
+    """Work list and repeated heads of one rank's share of the heads."""
+    rp = np.ascontiguousarray(row_ptr, np.int32)
+    mine = np.ascontiguousarray(np.asarray(owner) == rank, np.uint8)
+    rep = np.ascontiguousarray([int(h) for h in rep_heads if mine[int(h)]], np.int32)
+    nbq_b = -(-F * k_anchor * W // BLOCK)
+    out = np.empty(heads * nb + len(rep) * nbq_b, np.int32)
+    n = np.zeros(1, np.int32)
+    _check(load().calibatt_build_mixed_plan(_ptr(rp), heads, nb, _ptr(mine), len(rep), _ptr(rep) if len(rep) else None,
+                                            F, H, W, k_anchor, _ptr(out), _ptr(n)), "build_mixed_plan")
+    return out[: int(n[0])].copy(), rep.tolist()
 
 
 def anchor_rows(H: int, k_anchor: int) -> np.ndarray:

@@ -57,6 +57,11 @@ int check_qkv(const void* q, const void* k, const void* v, const void* o, int he
 
 bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 
+// Query blocks of the packed anchor queries of one repeated head.
+int64_t anchor_blocks(int frames, int W, int k_anchor) {
+  return (static_cast<int64_t>(frames) * k_anchor * W + 127) / 128;
+}
+
 KernelParams base_params() {
   KernelParams p;
   std::memset(&p, 0, sizeof p);
@@ -250,6 +255,35 @@ int calibatt_build_mixed_plan(const int32_t* row_ptr, int heads, int nb, const u
   return CALIBATT_OK;
 }
 
+int calibatt_shard_heads(const int32_t* row_ptr_host, int heads, int nb, const int32_t* rep_heads_host, int n_rep,
+                         int frames, int W, int k_anchor, int n_ranks, int32_t* owner, int64_t* load) {
+  if (!row_ptr_host || !owner || heads < 1 || nb < 1 || n_rep < 0 || n_rep > heads || (n_rep > 0 && !rep_heads_host) ||
+      frames < 1 || W < 1 || k_anchor < 1 || n_ranks < 1)
+    return CALIBATT_ERR_ARG;
+  std::vector<int64_t> cost(static_cast<size_t>(heads));
+  for (int h = 0; h < heads; ++h) {
+    const int64_t a = row_ptr_host[static_cast<int64_t>(h) * nb], b = row_ptr_host[static_cast<int64_t>(h + 1) * nb];
+    if (b < a) return CALIBATT_ERR_CSR;
+    cost[h] = b - a;
+  }
+  for (int i = 0; i < n_rep; ++i) {
+    const int h = rep_heads_host[i];
+    if (h < 0 || h >= heads) return CALIBATT_ERR_ARG;
+    cost[h] = anchor_blocks(frames, W, k_anchor) * nb;  // anchor-query tiles over every key block
+  }
+  std::vector<int> order(static_cast<size_t>(heads));
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  std::vector<int64_t> acc(static_cast<size_t>(n_ranks), 0);
+  for (int h : order) {
+    const int r = static_cast<int>(std::min_element(acc.begin(), acc.end()) - acc.begin());
+    owner[h] = r;
+    acc[r] += cost[h];
+  }
+  if (load) std::copy(acc.begin(), acc.end(), load);
+  return CALIBATT_OK;
+}
+
 int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v, int heads,
                             int frames, int H, int W, int d, int k_anchor, float scale, const int32_t* row_ptr,
                             const int32_t* col_idx, int64_t nnz, const int32_t* rep_heads, int32_t n_rep,
@@ -322,10 +356,6 @@ int host_pipe(int dev, int n_chunks, HostPipe** out) {
   }
   *out = &hp;
   return CALIBATT_OK;
-}
-
-int64_t anchor_blocks(int frames, int W, int k_anchor) {
-  return (static_cast<int64_t>(frames) * k_anchor * W + 127) / 128;
 }
 }  // namespace
 

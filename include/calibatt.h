@@ -170,6 +170,20 @@ int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, cons
                             const int32_t* work_list, int32_t n_work, calibatt_bf16* o, float* lse, void* ws,
                             size_t ws_bytes, calibatt_stream_t stream);
 
+/* Head sharding of one attention call over n_ranks GPUs (host). A head's
+ * output depends only on its own q, k, v, so ranks need no exchange; the
+ * work is balanced by kept tiles (a block-sparse head: its kept blocks; a
+ * repeated head: ceil(frames*k_anchor*W / 128) anchor blocks x nb): heads in
+ * descending cost (ties: lower head first), each to the least-loaded rank
+ * (ties: lower rank). Each rank then builds its work list with
+ * calibatt_build_mixed_plan, head_active[h] = (owner[h] == rank), and its
+ * own repeated heads.
+ *   row_ptr_host : host int32 [heads*nb + 1]; rep_heads_host: host int32 [n_rep]
+ *   owner        : host int32 [heads] (output: rank of each head)
+ *   load         : host int64 [n_ranks] (output: kept tiles per rank) or NULL */
+int calibatt_shard_heads(const int32_t* row_ptr_host, int heads, int nb, const int32_t* rep_heads_host, int n_rep,
+                         int frames, int W, int k_anchor, int n_ranks, int32_t* owner, int64_t* load);
+
 /* Device workspace bytes of calibatt_mixed_attn_fwd_host (anchor queries of
  * one chunk plus every chunk's work list); heads_per_chunk <= 0 means 2. */
 size_t calibatt_mixed_host_workspace_size(int heads, int frames, int H, int W, int k_anchor, int n_rep,

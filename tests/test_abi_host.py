@@ -214,6 +214,34 @@ def test_bank_index_on_the_host(binding):
     assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 8, P(0x100004), None) == -3
 
 
+def test_head_sharding_balances_and_partitions(binding, oracle):
+    from calibrated_block_sparse_b200 import synth
+    wl = synth.WORKLOADS["wan720"]
+    masks = synth.random_block_masks(wl)
+    row_ptr, _ = oracle.mask_to_csr(masks)
+    rep = list(wl.repeat_heads)
+    full = binding.build_mixed_plan(row_ptr, wl.heads, wl.nb, rep, wl.F, wl.H, wl.W)
+    cost = [int(row_ptr[(h + 1) * wl.nb] - row_ptr[h * wl.nb]) for h in range(wl.heads)]
+    for h in rep:
+        cost[h] = -(-wl.F * 5 * wl.W // 128) * wl.nb
+    for n_ranks in (1, 2, 4, 8):
+        owner, load = binding.shard_heads(row_ptr, wl.heads, wl.nb, rep, wl.F, wl.W, 5, n_ranks)
+        assert owner.min() >= 0 and owner.max() < n_ranks
+        np.testing.assert_array_equal(load, [sum(c for h, c in enumerate(cost) if owner[h] == r) for r in range(n_ranks)])
+        assert load.max() <= sum(cost) / n_ranks + max(cost)  # greedy longest-first bound
+        # the ranks' work lists partition the units of the whole call
+        units = []
+        for r in range(n_ranks):
+            w, rep_r = binding.build_rank_plan(row_ptr, wl.heads, wl.nb, rep, owner, r, wl.F, wl.H, wl.W)
+            assert all(owner[h] == r for h in rep_r)
+            nbq_b = -(-wl.F * 5 * wl.W // 128)
+            base = wl.heads * wl.nb
+            # anchor codes are local to the rank's repeated-head list: map them back
+            units += [int(u) if u < base else base + rep.index(rep_r[(u - base) // nbq_b]) * nbq_b + (u - base) % nbq_b
+                      for u in w]
+        assert sorted(units) == sorted(full.tolist())
+
+
 def test_workspace_sizes(binding):
     lib = binding.load()
     assert binding.repeat_workspace_size(8, 21, 45, 80, 5) == 8 * 21 * 5 * 80 * 256

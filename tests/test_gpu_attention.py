@@ -246,3 +246,34 @@ def test_host_buffer_pipeline_equals_device_call(oracle, chunk):
     assert binding.get_status() == 0
     assert torch.equal(oh, o_ref.cpu())
     assert torch.equal(lh, lse_ref.cpu())
+
+
+@pytest.mark.parametrize("n_ranks", [2, 3])
+def test_head_shards_together_equal_the_whole_call(oracle, n_ranks):
+    """The ranks' shares of one call (calibatt_shard_heads), run one after
+    another here, write bit for bit the output of the whole call."""
+    binding = require_gpu()
+    F, H, W, heads, kk = 3, 8, 16, 6, 5
+    n = F * H * W
+    nb = (n + 127) // 128
+    q, k, v = synth.plain_qkv(heads, n, seed=90 + n_ranks)
+    rng = np.random.default_rng(n_ranks)
+    mask = (rng.random((heads, nb, nb)) < rng.random((heads, 1, 1))).astype(np.uint8)
+    mask[:, np.arange(nb), np.arange(nb)] = 1
+    rep = [2, 5]
+    row_ptr, col_idx = oracle.mask_to_csr(mask)
+    dev = torch.device("cuda")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    rp_d, ci_d = torch.from_numpy(row_ptr).to(dev), torch.from_numpy(col_idx).to(dev)
+    work = torch.from_numpy(binding.build_mixed_plan(row_ptr, heads, nb, rep, F, H, W, kk)).to(dev)
+    o_all, lse_all = binding.mixed_attn_fwd(qd, kd, vd, F, H, W, rp_d, ci_d, torch.tensor(rep, dtype=torch.int32,
+                                                                                         device=dev), work, k_anchor=kk)
+    owner, _ = binding.shard_heads(row_ptr, heads, nb, rep, F, W, kk, n_ranks)
+    o = torch.zeros_like(qd)
+    lse = torch.zeros((heads, n), dtype=torch.float32, device=dev)
+    for r in range(n_ranks):
+        w, rep_r = binding.build_rank_plan(row_ptr, heads, nb, rep, owner, r, F, H, W, kk)
+        binding.mixed_attn_fwd(qd, kd, vd, F, H, W, rp_d, ci_d, torch.tensor(rep_r, dtype=torch.int32, device=dev),
+                               torch.from_numpy(w).to(dev), k_anchor=kk, o=o, lse=lse)
+    assert binding.get_status() == 0
+    assert torch.equal(o, o_all) and torch.equal(lse, lse_all)

@@ -72,3 +72,55 @@ def test_shard_range_partitions():
             assert all(a[1] == b[0] for a, b in zip(parts, parts[1:]))
             sizes = [hi - lo for lo, hi in parts]
             assert max(sizes) - min(sizes) <= 1
+
+
+def _plan_worker(rank, world, port, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from calibrated_block_sparse_b200 import binding, synth
+        wl = synth.WORKLOADS["mochi480"]
+        row_ptr, _ = oracle.mask_to_csr(synth.random_block_masks(wl))
+        rep = list(wl.repeat_heads)
+        owner, load = binding.shard_heads(row_ptr, wl.heads, wl.nb, rep, wl.F, wl.W, wl.k_anchor, world)
+        work, rep_r = binding.build_rank_plan(row_ptr, wl.heads, wl.nb, rep, owner, rank, wl.F, wl.H, wl.W)
+        # every rank derives the same owners on its own
+        owners = [torch.zeros(wl.heads, dtype=torch.int32) for _ in range(world)]
+        dist.all_gather(owners, torch.from_numpy(owner))
+        # the slowest rank's share of kept tiles
+        heaviest = torch.tensor([int(load[rank])], dtype=torch.int64)
+        dist.all_reduce(heaviest, op=dist.ReduceOp.MAX)
+        out_q.put((rank, [o.numpy() for o in owners], work, rep_r, int(heaviest.item()), load))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharding_over_two_ranks():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_plan_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = sorted([q.get(timeout=120) for _ in range(world)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, owners, _, _, heaviest, load in results:
+        np.testing.assert_array_equal(owners[0], owners[1])
+        assert heaviest == max(load)
+    owner = results[0][1][0]
+    for rank, _, work, rep_r, _, _ in results:
+        assert all(owner[h] == rank for h in rep_r)
+    # the two ranks' block-sparse units are disjoint and cover the sparse heads
+    from calibrated_block_sparse_b200 import synth
+    wl = synth.WORKLOADS["mochi480"]
+    base = wl.heads * wl.nb
+    sp = [set(int(u) for u in r[2] if u < base) for r in results]
+    assert not (sp[0] & sp[1])
+    assert sorted(sp[0] | sp[1]) == [h * wl.nb + r for h in range(wl.heads) if h not in wl.repeat_heads
+                                     for r in range(wl.nb)]
