@@ -20,15 +20,13 @@ template <int PER>
 __global__ void __launch_bounds__(128) select_kernel(const float* __restrict__ energy, int64_t rows, int nb,
                                                      long long eps_fx, uint8_t* mask, int32_t* kept,
                                                      uint16_t* counts) {
-  __shared__ float e_rows[4][1024];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + w;
   if (row >= rows) return;
-  const float* src = energy + row * nb;
-  for (int c = lane; c < nb; c += 32) e_rows[w][c] = src[c];
-  __syncwarp();
+  // each lane reads its own run of the row straight from global memory: the
+  // PER loads of a lane are independent and all in flight at once
   SelectOut out{mask ? mask + row * nb : nullptr, kept ? kept + row : nullptr, counts ? counts + row * nb : nullptr};
-  select_row<PER>(e_rows[w], nb, eps_fx, nullptr, lane, 32, 0, out);
+  select_row<PER>(energy + row * nb, nb, eps_fx, nullptr, lane, 32, 0, out);
 }
 
 // ------------------------------------------------------------------ accumulation

@@ -80,6 +80,19 @@ __device__ __forceinline__ void group_sum(long long& v, int& c, SelectScratch* s
   group_sync(bar_id, T);
 }
 
+// Sum of a per-thread int64 over the T threads (T multiple of 32).
+__device__ __forceinline__ long long group_sum64(long long v, SelectScratch* sc, int tid, int T, int bar_id) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (T == 32) return v;
+  if ((tid & 31) == 0) sc->wsum[tid >> 5] = v;
+  group_sync(bar_id, T);
+  v = 0;
+  for (int w = 0; w < (T >> 5); ++w) v += sc->wsum[w];
+  group_sync(bar_id, T);
+  return v;
+}
+
 // Max of a per-thread key over the T threads.
 __device__ __forceinline__ unsigned long long group_max(unsigned long long v, SelectScratch* sc, int tid, int T,
                                                         int bar_id) {
@@ -100,8 +113,8 @@ __device__ __forceinline__ unsigned long long group_max(unsigned long long v, Se
   return v;
 }
 
-// E: shared [nb] energies; aux: shared scratch of sizeof(SelectScratch)
-// (unused when T == 32). Every one of the T threads (T a multiple of 32,
+// E: [nb] energies (shared or global memory); aux: shared scratch of
+// sizeof(SelectScratch) (unused when T == 32). Every one of the T threads (T a multiple of 32,
 // nb <= PER * T) must call this. Thread tid owns columns tid*per .. +per-1.
 template <int PER>
 __device__ __forceinline__ void select_row(const float* E, int nb, long long eps_fx, uint8_t* aux, int tid, int T,
@@ -146,21 +159,22 @@ __device__ __forceinline__ void select_row(const float* E, int nb, long long eps
     uint32_t lo = 0, hi = top_bits;
     while (lo < hi) {
       const uint32_t mid = lo + (hi - lo + 1) / 2;
-      long long sm = 0;
-      int dummy = 0;
+      long long s0 = 0, s1 = 0;  // two chains: half the add latency
 #pragma unroll
-      for (int i = 0; i < PER; ++i) sm += bits[i] >= mid ? fx[i] : 0;
-      group_sum(sm, dummy, sc, tid, T, bar_id);
+      for (int i = 0; i < PER; i += 2) {
+        s0 += bits[i] >= mid ? fx[i] : 0;
+        if (i + 1 < PER) s1 += bits[i + 1] >= mid ? fx[i + 1] : 0;
+      }
+      const long long sm = group_sum64(s0 + s1, sc, tid, T, bar_id);
       if (sm >= eps_fx)
         lo = mid;
       else
         hi = mid - 1;
     }
     tau = lo;
-    int dummy = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) above += bits[i] > tau ? fx[i] : 0;
-    group_sum(above, dummy, sc, tid, T, bar_id);
+    above = group_sum64(above, sc, tid, T, bar_id);
   }
 
   // rank of each block among the blocks equal to tau, in column order
