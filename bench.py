@@ -295,10 +295,12 @@ def run_ours(args, world, rank, local):
         # masks calibrated on the GPU over the workload's seeded inputs
         n_cal, eps_cal = synth.CALIBRATION[args.workload]
         counts = torch.zeros((heads, nb, nb), dtype=torch.uint16, device=dev)
+        cws = torch.empty(binding.energy_workspace_size(heads, n), dtype=torch.uint8, device=dev)
         for pi in range(n_cal):
             qc, kc, _ = synth.qkv(wl, pi, with_v=False, device=dev)
-            binding.block_energy(qc, kc, eps=eps_cal, energy=False, counts=counts)
+            binding.block_energy_1pass(qc, kc, eps=eps_cal, energy=False, counts=counts, ws=cws)
             del qc, kc
+        del cws
         mask_d, row_ptr, col_idx, _ = binding.aggregate_masks(counts, n_cal, 0.5)
         masks = mask_d.cpu().numpy()
     binding.check_status(what="skip lists")

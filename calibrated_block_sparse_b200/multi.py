@@ -51,7 +51,7 @@ def calibrate_sharded(inputs, heads: int, nb: int, n_inputs: int, eps: float, rh
     """Calibrate one (t, l) over n_inputs inputs split across the ranks.
 
     ``inputs(p)`` returns (q, k) bf16 CUDA tensors of input p. Each rank runs
-    the fused block-energy + greedy-selection kernel on its share, the counts
+    the single-pass block-energy + greedy-selection kernel on its share, the counts
     are summed over ranks, and the aggregated mask and skip list are built on
     every rank. Returns (mask, row_ptr, col_idx, nnz)."""
     from . import binding
@@ -59,9 +59,13 @@ def calibrate_sharded(inputs, heads: int, nb: int, n_inputs: int, eps: float, rh
     world = dist.get_world_size(group) if dist.is_initialized() else 1
     lo, hi = shard_range(n_inputs, rank, world)
     counts = torch.zeros((heads, nb, nb), dtype=torch.uint16, device=device)
+    ws = None
     for p in range(lo, hi):
         q, k = inputs(p)
-        binding.block_energy(q, k, eps=eps, energy=False, counts=counts)
+        if ws is None:  # single-pass energy: one S per tile; workspace reused over inputs
+            ws = torch.empty(binding.energy_workspace_size(q.shape[0], q.shape[1]), dtype=torch.uint8,
+                             device=q.device)
+        binding.block_energy_1pass(q, k, eps=eps, energy=False, counts=counts, ws=ws)
     binding.check_status(what="calibration")
     if world > 1:
         allreduce_counts(counts, group)
