@@ -174,9 +174,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const uint64_t kdesc0 = desc_k_base(sbase + L::kRingOff);
     while (true) {
       if (!mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status)) break;
+      // read every word of the stage now: once ring_empty is committed below,
+      // the producer may reuse the stage and rewrite them for its next tile
       const uint32_t s = *reinterpret_cast<volatile uint32_t*>(&bar.slot[stage]);
       if (s > 1) break;
-      if (*reinterpret_cast<volatile uint32_t*>(&bar.first[stage])) {
+      const bool first = *reinterpret_cast<volatile uint32_t*>(&bar.first[stage]) != 0;
+      const bool last = *reinterpret_cast<volatile uint32_t*>(&bar.last[stage]) != 0;
+      if (first) {
         if (!mbar_wait(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status)) break;
       }
       const int buf = n_s[s] & 1;
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) mma_ss(d_tmem, qd + desc_k_step(ks), kd + desc_k_step(ks), kIdescS, ks > 0);
       mma_commit(&bar.ring_empty[stage]);
-      if (*reinterpret_cast<volatile uint32_t*>(&bar.last[stage])) {
+      if (last) {
         mma_commit(&bar.q_empty[s]);
         ++n_q[s];
       }
