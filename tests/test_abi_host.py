@@ -26,7 +26,7 @@ def _declared():
     return sorted(set(re.findall(r"\b(calibatt_[a-z0-9_]+)\s*\(", text)))
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_hot_path_calls():
     names = _declared()
     for n in ("calibatt_block_energy", "calibatt_select_mask", "calibatt_aggregate_masks",
               "calibatt_sparse_attn_fwd", "calibatt_repeat_attn_fwd"):
