@@ -277,3 +277,41 @@ def test_head_shards_together_equal_the_whole_call(oracle, n_ranks):
                                torch.from_numpy(w).to(dev), k_anchor=kk, o=o, lse=lse)
     assert binding.get_status() == 0
     assert torch.equal(o, o_all) and torch.equal(lse, lse_all)
+
+
+def test_mixed_launch_edge_cases(oracle):
+    """Every head repeated (no block-sparse unit); an empty work list (nothing
+    written); a host-buffer chunk larger than the head count."""
+    binding = require_gpu()
+    F, H, W, heads, kk = 2, 8, 16, 3, 5
+    n = F * H * W
+    nb = (n + 127) // 128
+    q, k, v = synth.plain_qkv(heads, n, seed=77)
+    dev = torch.device("cuda")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    mask = np.ones((heads, nb, nb), np.uint8)
+    row_ptr, col_idx = oracle.mask_to_csr(mask)
+    rp_d, ci_d = torch.from_numpy(row_ptr).to(dev), torch.from_numpy(col_idx).to(dev)
+    rep = [0, 1, 2]
+    rep_d = torch.tensor(rep, dtype=torch.int32, device=dev)
+    work = binding.build_mixed_plan(row_ptr, heads, nb, rep, F, H, W, kk)
+    assert work.min() >= heads * nb  # anchor-query units only
+    o, _ = binding.mixed_attn_fwd(qd, kd, vd, F, H, W, rp_d, ci_d, rep_d, torch.from_numpy(work).to(dev), k_anchor=kk)
+    o_ref, _ = oracle.repeat_attention(synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v), F, H, W,
+                                       k_anchor=kk)
+    assert attn_tolerance_ok(bf16_to_f64(o), o_ref)[0]
+    # an empty work list writes nothing
+    o2 = torch.full_like(qd, 3.0)
+    binding.mixed_attn_fwd(qd, kd, vd, F, H, W, rp_d, ci_d, torch.zeros(0, dtype=torch.int32, device=dev),
+                           torch.zeros(0, dtype=torch.int32, device=dev), k_anchor=kk, o=o2)
+    assert binding.get_status() == 0
+    assert bool((o2 == 3.0).all())
+    # host buffers with one chunk holding every head
+    qh, kh, vh = (t.contiguous().pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(q).pin_memory()
+    bufs = [torch.empty_like(qd) for _ in range(4)]
+    binding.mixed_attn_fwd_host(qh, kh, vh, oh, F, H, W, row_ptr, rp_d, ci_d, rep, *bufs, heads_per_chunk=16,
+                                k_anchor=kk)
+    torch.cuda.synchronize()
+    assert binding.get_status() == 0
+    assert torch.equal(oh, o.cpu())

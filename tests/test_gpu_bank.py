@@ -51,6 +51,7 @@ def test_calibrate_into_bank_then_infer_by_lookup(oracle):
             hist = binding.keep_histogram(counts, N_IN).cpu().numpy()
             c_host = counts.view(torch.int16).cpu().numpy().astype(np.int64) & 0xFFFF
             np.testing.assert_array_equal(hist, oracle.keep_histogram(c_host, N_IN))
+            np.testing.assert_array_equal((hist * np.arange(N_IN + 1)).sum(-1), c_host.sum(axis=(1, 2)))
             mask, row_ptr, col_idx, _ = binding.aggregate_masks(counts, N_IN, 0.5)
             bank.put(t, l, eps_t, row_ptr, col_idx, rep)
             stored[(t, l)] = (wl, eps_t, mask.cpu().numpy(), row_ptr.cpu().numpy(), col_idx.cpu().numpy(), rep)
@@ -101,3 +102,11 @@ def test_keep_histogram_matches_oracle_and_reports_bad_counts(oracle):
     hist = binding.keep_histogram(bad, n_in).cpu().numpy()
     assert binding.get_status() == -1   # reported ...
     assert hist[0].sum() == 591 * 591   # ... and counted in the last bin
+
+
+def test_bank_lookup_of_a_missing_entry_raises():
+    binding = require_gpu()
+    bank = binding.MaskBank(2, 2, 1, 2, 8, 16, 5)
+    with pytest.raises(binding.CalibattError):
+        bank.get(1, 1)
+    bank.close()
