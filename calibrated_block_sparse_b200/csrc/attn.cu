@@ -2,13 +2,17 @@
 // repeated heads, on the sm_100a tensor core (explainer §三, online
 // inference): O = softmax(scale Q K^T) V over the kept 128 x 128 tiles.
 //
-// CTA (320 threads, one per SM, persistent over a longest-first unit list),
+// CTA (384 threads, one per SM, persistent over a longest-first unit list),
 // two independent query-tile "slots" so that the tensor core works on one
 // slot while the other slot's softmax runs:
 //   warps 0-3  softmax warpgroup of slot 0 (thread = query row = TMEM lane)
 //   warps 4-7  softmax warpgroup of slot 1
 //   warp  8    TMA producer (one thread): Q tile per unit, K/V tiles per kept block
 //   warp  9    MMA issuer (one thread): tcgen05.mma S = Q K^T and O += P V
+//   warps 10-11 idle (they complete the third warpgroup)
+// The third warpgroup hands registers to the softmax warpgroups (setmaxnreg):
+// a softmax thread holds a whole 128-column row of S, and at the launch
+// allotment of 168 registers it spilled.
 // Tensor memory (512 columns): S (fp32, 128 columns) and O (fp32, 128
 // columns) per slot; P (bf16) is written over the first 64 columns of S and
 // read by the P V MMA from there. The MMA issue order merges the two slots'
@@ -35,7 +39,12 @@
 namespace calibatt {
 namespace {
 
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;
+constexpr int kSoftmaxRegs = 200;  // warps 0-7 after the split
+constexpr int kControlRegs = 96;   // warps 8-11 after the split
+// the split must fit in the launch allotment (checked against the compiled
+// kernel's count before every launch): 168 registers x 384 threads
+static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= 168 * kAttnThreads, "register split");
 constexpr int kAttnRing = 5;               // K/V tiles in flight
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: move the running max only if it grows by more
 
@@ -97,138 +106,142 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
 
-  if (warp == 8 && lane == 0) {
-    // ---------------------------------------------------------- TMA producer
-    tma_prefetch_desc(&tm_q);
-    if (p.nbq_b > 0) tma_prefetch_desc(&tm_qb);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    Cursor cur[2];
-    for (int s = 0; s < 2; ++s) {
-      cur[s].round = 0;
-      cursor_seek(p, 2 * blockIdx.x + s, G, cur[s]);
-    }
-    uint32_t stage = 0, phase = 0, n_q[2] = {0, 0};
-    bool ok = true;
-    auto load_tile = [&](const CUtensorMap* map, int blk, int head) -> bool {
-      if (!mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status)) return false;
-      uint8_t* dst = smem + L::kRingOff + stage * kTile;
-      mbar_arrive_expect_tx(&bar.ring_full[stage], kTile);
-      tma_load_3d(dst, map, &bar.ring_full[stage], 0, blk * 128, head);
-      tma_load_3d(dst + kHalf, map, &bar.ring_full[stage], 64, blk * 128, head);
-      if (++stage == kAttnRing) {
-        stage = 0;
-        phase ^= 1;
+  if (warp >= 8) {
+    warpgroup_regs_dec<kControlRegs>();
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      tma_prefetch_desc(&tm_q);
+      if (p.nbq_b > 0) tma_prefetch_desc(&tm_qb);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      Cursor cur[2];
+      for (int s = 0; s < 2; ++s) {
+        cur[s].round = 0;
+        cursor_seek(p, 2 * blockIdx.x + s, G, cur[s]);
       }
-      return true;
-    };
-    auto emit_s = [&](int s) -> bool {
-      Cursor& c = cur[s];
-      if (c.j == 0) {
-        if (!mbar_wait(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status)) return false;
-        uint8_t* dst = smem + L::kQOff + s * kTile;
-        const CUtensorMap* qmap = c.u.rep ? &tm_qb : &tm_q;
-        mbar_arrive_expect_tx(&bar.q_full[s], kTile);
-        tma_load_3d(dst, qmap, &bar.q_full[s], 0, c.u.r * 128, c.u.hq);
-        tma_load_3d(dst + kHalf, qmap, &bar.q_full[s], 64, c.u.r * 128, c.u.hq);
-        ++n_q[s];
-      }
-      return load_tile(&tm_k, block_col(p, c.u, c.j), c.u.hkv);
-    };
-    for (int s = 0; s < 2 && ok; ++s)
-      if (cur[s].valid) ok = emit_s(s);
-    while (ok && (cur[0].valid || cur[1].valid)) {
-      for (int s = 0; s < 2 && ok; ++s) {
-        if (!cur[s].valid) continue;
-        ok = load_tile(&tm_v, block_col(p, cur[s].u, cur[s].j), cur[s].u.hkv);
-        if (!ok) break;
-        cursor_next(p, 2 * blockIdx.x + s, G, cur[s]);
+      uint32_t stage = 0, phase = 0, n_q[2] = {0, 0};
+      bool ok = true;
+      auto load_tile = [&](const CUtensorMap* map, int blk, int head) -> bool {
+        if (!mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status)) return false;
+        uint8_t* dst = smem + L::kRingOff + stage * kTile;
+        mbar_arrive_expect_tx(&bar.ring_full[stage], kTile);
+        tma_load_3d(dst, map, &bar.ring_full[stage], 0, blk * 128, head);
+        tma_load_3d(dst + kHalf, map, &bar.ring_full[stage], 64, blk * 128, head);
+        if (++stage == kAttnRing) {
+          stage = 0;
+          phase ^= 1;
+        }
+        return true;
+      };
+      auto emit_s = [&](int s) -> bool {
+        Cursor& c = cur[s];
+        if (c.j == 0) {
+          if (!mbar_wait(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status)) return false;
+          uint8_t* dst = smem + L::kQOff + s * kTile;
+          const CUtensorMap* qmap = c.u.rep ? &tm_qb : &tm_q;
+          mbar_arrive_expect_tx(&bar.q_full[s], kTile);
+          tma_load_3d(dst, qmap, &bar.q_full[s], 0, c.u.r * 128, c.u.hq);
+          tma_load_3d(dst + kHalf, qmap, &bar.q_full[s], 64, c.u.r * 128, c.u.hq);
+          ++n_q[s];
+        }
+        return load_tile(&tm_k, block_col(p, c.u, c.j), c.u.hkv);
+      };
+      for (int s = 0; s < 2 && ok; ++s)
         if (cur[s].valid) ok = emit_s(s);
+      while (ok && (cur[0].valid || cur[1].valid)) {
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (!cur[s].valid) continue;
+          ok = load_tile(&tm_v, block_col(p, cur[s].u, cur[s].j), cur[s].u.hkv);
+          if (!ok) break;
+          cursor_next(p, 2 * blockIdx.x + s, G, cur[s]);
+          if (cur[s].valid) ok = emit_s(s);
+        }
       }
-    }
-    // no copy may still be landing when the CTA leaves: the latest load of
-    // every ring stage and Q buffer has completed
-    for (int i = 0; i < kAttnRing; ++i) {
-      int st = static_cast<int>(stage) - 1 - i;
-      uint32_t ph = phase;
-      if (st < 0) {
-        st += kAttnRing;
-        ph ^= 1;
-      }
-      volatile int never = 0;
-      mbar_wait(&bar.ring_full[st], ph, &never, p.status);
-    }
-    for (int s = 0; s < 2; ++s)
-      if (n_q[s] > 0) {
+      // no copy may still be landing when the CTA leaves: the latest load of
+      // every ring stage and Q buffer has completed
+      for (int i = 0; i < kAttnRing; ++i) {
+        int st = static_cast<int>(stage) - 1 - i;
+        uint32_t ph = phase;
+        if (st < 0) {
+          st += kAttnRing;
+          ph ^= 1;
+        }
         volatile int never = 0;
-        mbar_wait(&bar.q_full[s], (n_q[s] - 1) & 1, &never, p.status);
+        mbar_wait(&bar.ring_full[st], ph, &never, p.status);
       }
-  } else if (warp == 9 && lane == 0) {
-    // ---------------------------------------------------------- MMA issuer
-    Cursor cur[2];
-    for (int s = 0; s < 2; ++s) {
-      cur[s].round = 0;
-      cursor_seek(p, 2 * blockIdx.x + s, G, cur[s]);
-    }
-    uint32_t stage = 0, phase = 0, n_q[2] = {0, 0}, n_pv[2] = {0, 0};
-    const uint64_t qdesc0 = desc_k_base(sbase + L::kQOff);
-    const uint64_t kdesc0 = desc_k_base(sbase + L::kRingOff);
-    const uint64_t vdesc0 = desc_v_base(sbase + L::kRingOff);
-    bool ok = true;
-    auto next_stage = [&]() {
-      if (++stage == kAttnRing) {
-        stage = 0;
-        phase ^= 1;
+      for (int s = 0; s < 2; ++s)
+        if (n_q[s] > 0) {
+          volatile int never = 0;
+          mbar_wait(&bar.q_full[s], (n_q[s] - 1) & 1, &never, p.status);
+        }
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      Cursor cur[2];
+      for (int s = 0; s < 2; ++s) {
+        cur[s].round = 0;
+        cursor_seek(p, 2 * blockIdx.x + s, G, cur[s]);
       }
-    };
-    auto issue_s = [&](int s) -> bool {
-      Cursor& c = cur[s];
-      if (c.j == 0) {
-        if (!mbar_wait(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status)) return false;
-      }
-      if (!mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status)) return false;
-      tc_fence_after();
-      const uint64_t qd = qdesc0 + s * (kTile >> 4), kd = kdesc0 + stage * (kTile >> 4);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_ss(tmem + s * 128, qd + desc_k_step(ks), kd + desc_k_step(ks), kIdescS, ks > 0);
-      mma_commit(&bar.ring_empty[stage]);
-      if (c.j == c.u.nnz - 1) {
-        mma_commit(&bar.q_empty[s]);
-        ++n_q[s];
-      }
-      mma_commit(&bar.s_full[s]);
-      next_stage();
-      return true;
-    };
-    for (int s = 0; s < 2 && ok; ++s)
-      if (cur[s].valid) ok = issue_s(s);
-    while (ok && (cur[0].valid || cur[1].valid)) {
-      for (int s = 0; s < 2 && ok; ++s) {
-        if (!cur[s].valid) continue;
-        // O += P V for the current block of slot s (P read from tensor memory)
-        if (!(ok = mbar_wait(&bar.p_full[s], n_pv[s] & 1, abort_flag, p.status))) break;
-        if (!(ok = mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status))) break;
+      uint32_t stage = 0, phase = 0, n_q[2] = {0, 0}, n_pv[2] = {0, 0};
+      const uint64_t qdesc0 = desc_k_base(sbase + L::kQOff);
+      const uint64_t kdesc0 = desc_k_base(sbase + L::kRingOff);
+      const uint64_t vdesc0 = desc_v_base(sbase + L::kRingOff);
+      bool ok = true;
+      auto next_stage = [&]() {
+        if (++stage == kAttnRing) {
+          stage = 0;
+          phase ^= 1;
+        }
+      };
+      auto issue_s = [&](int s) -> bool {
+        Cursor& c = cur[s];
+        if (c.j == 0) {
+          if (!mbar_wait(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status)) return false;
+        }
+        if (!mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint64_t vd = vdesc0 + stage * (kTile >> 4);
+        const uint64_t qd = qdesc0 + s * (kTile >> 4), kd = kdesc0 + stage * (kTile >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ts(tmem + 256 + s * 128, tmem + s * 128 + ks * 8, vd + desc_v_step(ks), kIdescPV,
-                 (cur[s].j > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(tmem + s * 128, qd + desc_k_step(ks), kd + desc_k_step(ks), kIdescS, ks > 0);
         mma_commit(&bar.ring_empty[stage]);
-        if (cur[s].j == cur[s].u.nnz - 1) mma_commit(&bar.o_full[s]);
-        ++n_pv[s];
+        if (c.j == c.u.nnz - 1) {
+          mma_commit(&bar.q_empty[s]);
+          ++n_q[s];
+        }
+        mma_commit(&bar.s_full[s]);
         next_stage();
-        cursor_next(p, 2 * blockIdx.x + s, G, cur[s]);
+        return true;
+      };
+      for (int s = 0; s < 2 && ok; ++s)
         if (cur[s].valid) ok = issue_s(s);
+      while (ok && (cur[0].valid || cur[1].valid)) {
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (!cur[s].valid) continue;
+          // O += P V for the current block of slot s (P read from tensor memory)
+          if (!(ok = mbar_wait(&bar.p_full[s], n_pv[s] & 1, abort_flag, p.status))) break;
+          if (!(ok = mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint64_t vd = vdesc0 + stage * (kTile >> 4);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ts(tmem + 256 + s * 128, tmem + s * 128 + ks * 8, vd + desc_v_step(ks), kIdescPV,
+                   (cur[s].j > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&bar.ring_empty[stage]);
+          if (cur[s].j == cur[s].u.nnz - 1) mma_commit(&bar.o_full[s]);
+          ++n_pv[s];
+          next_stage();
+          cursor_next(p, 2 * blockIdx.x + s, G, cur[s]);
+          if (cur[s].valid) ok = issue_s(s);
+        }
       }
+      // every issued MMA has finished before tensor memory is released
+      mma_commit(&bar.mma_done);
+      volatile int never = 0;
+      mbar_wait(&bar.mma_done, 0, &never, p.status);
     }
-    // every issued MMA has finished before tensor memory is released
-    mma_commit(&bar.mma_done);
-    volatile int never = 0;
-    mbar_wait(&bar.mma_done, 0, &never, p.status);
-  } else if (warp < 8) {
+  } else {
     // ---------------------------------------------------------- softmax warpgroups
+    warpgroup_regs_inc<kSoftmaxRegs>();
     // After a failed wait the warps keep walking their units with every wait
     // and tensor-memory access skipped, so that the CTA still reaches its
     // final barrier.
@@ -384,6 +397,14 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mqb, const CUtensorMap
       return CALIBATT_ERR_CUDA;
     configured = true;
   }
+  // the register split needs the allotment it was sized for
+  static int launch_regs = 0;
+  if (launch_regs == 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_kernel) != cudaSuccess) return CALIBATT_ERR_CUDA;
+    launch_regs = fa.numRegs;
+  }
+  if (launch_regs * kAttnThreads < 256 * kSoftmaxRegs + 128 * kControlRegs) return CALIBATT_ERR_CUDA;
   if (p.n_units <= 0) return CALIBATT_OK;
   int grid = (p.n_units + 1) / 2;
   const int sms = sm_count();

@@ -96,6 +96,21 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// ------------------------------------------------------------------ registers
+// Per-warpgroup register budget (every warp of the warpgroup executes it).
+// An increase waits until enough registers of the CTA's launch allotment
+// (threads x registers per thread at launch) have been released by decreases.
+template <int N>
+__device__ __forceinline__ void warpgroup_regs_dec() {
+  static_assert(N >= 24 && N <= 256 && N % 8 == 0, "register count");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void warpgroup_regs_inc() {
+  static_assert(N >= 24 && N <= 256 && N % 8 == 0, "register count");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
