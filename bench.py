@@ -419,7 +419,9 @@ def run_ours(args, world, rank, local):
         e2e_ms = max_over_ranks(cuda_time(e2e_step, reps, stream), world)
         binding.check_status(what="e2e")
         e2e = {"value": world * f_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()),
+               # q of a repeated head: its anchor pixel rows only
+               "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()
+                                         - len(rep_heads) * wl.F * (wl.H - wl.k_anchor) * wl.W * D * 2),
                "d2h_bytes_per_step": int(o.numel() * o.element_size()), "ms_per_step": e2e_ms,
                "call": f"calibatt_mixed_attn_fwd_host, pinned host buffers, {args.e2e_chunk} heads per chunk"}
         del qh, kh, vh, oh, ws_host

@@ -395,8 +395,13 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
   const int hpc = heads_per_chunk > 0 ? std::min(heads_per_chunk, heads) : std::min(2, heads);
   const int n_chunks = (heads + hpc - 1) / hpc;
   const int64_t nbq_b = anchor_blocks(frames, W, k_anchor);
-  for (int i = 0; i < n_rep; ++i)
+  std::vector<uint8_t> is_rep(static_cast<size_t>(heads), 0);
+  for (int i = 0; i < n_rep; ++i) {
     if (rep_heads_host[i] < 0 || rep_heads_host[i] >= heads) return CALIBATT_ERR_ARG;
+    is_rep[rep_heads_host[i]] = 1;
+  }
+  std::vector<int32_t> anchors(static_cast<size_t>(k_anchor));
+  calibatt_anchor_rows(H, k_anchor, anchors.data());
   // every chunk's work list and repeated heads, staged to the device in one
   // copy before any launch (a later pageable copy could wait for the stream)
   std::vector<int32_t> lists;
@@ -443,8 +448,30 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
     const int h0 = c * hpc, h1 = std::min(heads, h0 + hpc);
     const size_t off = static_cast<size_t>(h0) * head_elems, cnt = static_cast<size_t>(h1 - h0) * head_elems * 2;
     cudaEvent_t ev_in = hp->ev[2 + 2 * c], ev_done = hp->ev[3 + 2 * c];
-    if (!ok(cudaMemcpyAsync(q_dev + off, q_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
-        !ok(cudaMemcpyAsync(k_dev + off, k_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
+    // q: runs of whole heads; a repeated head reads only its anchor pixel rows,
+    // so only those are copied (one strided copy per anchor row: one W-token
+    // row of every frame)
+    for (int h = h0; h < h1;) {
+      if (is_rep[h]) {
+        const size_t frame_bytes = static_cast<size_t>(H) * W * 128 * 2, row_bytes = static_cast<size_t>(W) * 128 * 2;
+        for (int j = 0; j < k_anchor; ++j) {
+          const size_t e0 = (static_cast<size_t>(h) * n + static_cast<size_t>(anchors[j]) * W) * 128;
+          if (!ok(cudaMemcpy2DAsync(q_dev + e0, frame_bytes, q_host + e0, frame_bytes, row_bytes, frames,
+                                    cudaMemcpyHostToDevice, hp->in)))
+            return CALIBATT_ERR_CUDA;
+        }
+        ++h;
+      } else {
+        int e = h;
+        while (e < h1 && !is_rep[e]) ++e;
+        const size_t o0 = static_cast<size_t>(h) * head_elems;
+        if (!ok(cudaMemcpyAsync(q_dev + o0, q_host + o0, static_cast<size_t>(e - h) * head_elems * 2,
+                                cudaMemcpyHostToDevice, hp->in)))
+          return CALIBATT_ERR_CUDA;
+        h = e;
+      }
+    }
+    if (!ok(cudaMemcpyAsync(k_dev + off, k_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
         !ok(cudaMemcpyAsync(v_dev + off, v_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
         !ok(cudaEventRecord(ev_in, hp->in)) || !ok(cudaStreamWaitEvent(st, ev_in, 0)))
       return CALIBATT_ERR_CUDA;

@@ -198,7 +198,9 @@ size_t calibatt_mixed_host_workspace_size(int heads, int frames, int H, int W, i
  * when `stream` completes. Use page-locked host memory, else the copies do not
  * overlap. The skip list, work lists and repeated heads are those of
  * calibatt_mixed_attn_fwd; the work list of each chunk is built here from
- * row_ptr_host.
+ * row_ptr_host. Of a repeated head's q only the anchor pixel rows are copied
+ * (its other rows of q_dev are neither read nor written): the in-copy per step
+ * is 3*heads*n*256 bytes less n_rep*frames*(H - k_anchor)*W*256.
  *   q_host, k_host, v_host : host bf16 [heads][n][128]; o_host: host bf16 (output)
  *   lse_host  : host fp32 [heads][n] or NULL (then lse_dev may be NULL)
  *   row_ptr_host : host int32 [heads*nb + 1]; row_ptr, col_idx: the same list on the device

@@ -218,7 +218,9 @@ def test_mixed_launch_without_repeated_heads_is_the_sparse_call(oracle):
 @pytest.mark.parametrize("chunk", [1, 2, 8])
 def test_host_buffer_pipeline_equals_device_call(oracle, chunk):
     """calibatt_mixed_attn_fwd_host (copies in, compute, copies out, pipelined
-    over chunks of heads) returns bit for bit the device call's o and lse."""
+    over chunks of heads) returns bit for bit the device call's o and lse; of
+    a repeated head's q it copies the anchor pixel rows only and leaves the
+    other rows of the device buffer as they were."""
     binding = require_gpu()
     F, H, W, heads, kk = 3, 8, 16, 5, 5
     n = F * H * W
@@ -239,6 +241,7 @@ def test_host_buffer_pipeline_equals_device_call(oracle, chunk):
     oh = torch.empty_like(q).pin_memory()
     lh = torch.empty((heads, n), dtype=torch.float32).pin_memory()
     qd, kd, vd, od = (torch.empty_like(q, device=dev) for _ in range(4))
+    qd.fill_(float("nan"))
     ld = torch.empty((heads, n), dtype=torch.float32, device=dev)
     binding.mixed_attn_fwd_host(qh, kh, vh, oh, F, H, W, row_ptr, rp_d, ci_d, rep, qd, kd, vd, od, lse_host=lh,
                                 lse_dev=ld, heads_per_chunk=chunk, k_anchor=kk)
@@ -246,6 +249,16 @@ def test_host_buffer_pipeline_equals_device_call(oracle, chunk):
     assert binding.get_status() == 0
     assert torch.equal(oh, o_ref.cpu())
     assert torch.equal(lh, lse_ref.cpu())
+    anchors = oracle.anchor_rows(H, kk)
+    rows = (np.arange(n) // W) % H
+    copied = np.isin(rows, anchors)
+    qd_h = qd.cpu()
+    for h in range(heads):
+        if h in rep:
+            assert torch.equal(qd_h[h, torch.from_numpy(copied)], q[h, torch.from_numpy(copied)])
+            assert bool(torch.isnan(qd_h[h, torch.from_numpy(~copied)].float()).all())
+        else:
+            assert torch.equal(qd_h[h], q[h])
 
 
 @pytest.mark.parametrize("n_ranks", [2, 3])
