@@ -418,12 +418,27 @@ def run_ours(args, world, rank, local):
         barrier(world)
         e2e_ms = max_over_ranks(cuda_time(e2e_step, reps, stream), world)
         binding.check_status(what="e2e")
+
+        # the host link on its own: the same pinned q, k, v copied in whole
+        # with plain copies, no compute (the bound of the call above)
+        def link_step():
+            with torch.cuda.stream(stream):
+                q.copy_(qh, non_blocking=True)
+                k.copy_(kh, non_blocking=True)
+                v.copy_(vh, non_blocking=True)
+
+        link_step()
+        link_ms = cuda_time(link_step, reps, stream)
+        link_gbs = 3 * q.numel() * q.element_size() / (link_ms * 1e-3) / 1e9
         e2e = {"value": world * f_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                # q of a repeated head: its anchor pixel rows only
                "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()
                                          - len(rep_heads) * wl.F * (wl.H - wl.k_anchor) * wl.W * D * 2),
                "d2h_bytes_per_step": int(o.numel() * o.element_size()), "ms_per_step": e2e_ms,
+               "h2d_link_gbs": link_gbs,
                "call": f"calibatt_mixed_attn_fwd_host, pinned host buffers, {args.e2e_chunk} heads per chunk"}
+        # share of the link's copy-in rate that the call sustains
+        e2e["h2d_link_frac"] = e2e["h2d_bytes_per_step"] / (e2e_ms * 1e-3) / 1e9 / link_gbs
         del qh, kh, vh, oh, ws_host
 
     # ---- calibration kernels on the same shape (8 heads of it)
