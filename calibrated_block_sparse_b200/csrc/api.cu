@@ -333,10 +333,12 @@ int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, cons
 
 // ------------------------------------------------------------------ host buffers
 // Streams and events of the host-buffer pipeline, created once per device
-// (copies in and out overlap the caller's compute stream).
+// (copies in and out overlap the attention; odd chunks' attention runs on a
+// second compute stream, so that one chunk's launch fills the SMs that the
+// previous chunk's last units leave idle).
 namespace {
 struct HostPipe {
-  cudaStream_t in = nullptr, out = nullptr;
+  cudaStream_t in = nullptr, out = nullptr, cmp = nullptr;
   std::vector<cudaEvent_t> ev;  // [start, end, in_0, done_0, in_1, done_1, ...]
 };
 
@@ -347,7 +349,8 @@ int host_pipe(int dev, int n_chunks, HostPipe** out) {
   static HostPipe pipes[64];
   HostPipe& hp = pipes[dev];
   if (!hp.in && (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
-                 cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess))
+                 cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess ||
+                 cudaStreamCreateWithFlags(&hp.cmp, cudaStreamNonBlocking) != cudaSuccess))
     return CALIBATT_ERR_CUDA;
   while (static_cast<int>(hp.ev.size()) < 2 + 2 * n_chunks) {
     cudaEvent_t e;
@@ -366,9 +369,10 @@ size_t calibatt_mixed_host_workspace_size(int heads, int frames, int H, int W, i
   const int hpc = heads_per_chunk > 0 ? std::min(heads_per_chunk, heads) : std::min(2, heads);
   const int64_t n = static_cast<int64_t>(frames) * H * W;
   const int64_t nb = (n + 127) / 128;
+  // two anchor buffers (consecutive chunks may run at once), then the lists
   const size_t anchors = n_rep > 0 ? calibatt_repeat_workspace_size(std::min(hpc, n_rep), frames, H, W, k_anchor) : 0;
   const size_t lists = static_cast<size_t>(heads * nb + n_rep * anchor_blocks(frames, W, k_anchor) + n_rep) * 4;
-  return ((anchors + 255) & ~static_cast<size_t>(255)) + ((lists + 255) & ~static_cast<size_t>(255));
+  return 2 * ((anchors + 255) & ~static_cast<size_t>(255)) + ((lists + 255) & ~static_cast<size_t>(255));
 }
 
 int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf16* k_host,
@@ -393,7 +397,13 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
   if (!aligned16(ws) || (lse_dev && !aligned4(lse_dev))) return CALIBATT_ERR_ALIGN;
   const int nb = (n + 127) / 128;
   const int hpc = heads_per_chunk > 0 ? std::min(heads_per_chunk, heads) : std::min(2, heads);
-  const int n_chunks = (heads + hpc - 1) / hpc;
+  // chunk boundaries: the first chunk holds half as many heads (rounded up),
+  // so that the one copy-in that no attention overlaps is short; then chunks
+  // of hpc heads, the last one what remains
+  std::vector<int> bound{0};
+  if (hpc < heads) bound.push_back((hpc + 1) / 2);
+  while (bound.back() < heads) bound.push_back(std::min(heads, bound.back() + hpc));
+  const int n_chunks = static_cast<int>(bound.size()) - 1;
   const int64_t nbq_b = anchor_blocks(frames, W, k_anchor);
   std::vector<uint8_t> is_rep(static_cast<size_t>(heads), 0);
   for (int i = 0; i < n_rep; ++i) {
@@ -409,7 +419,7 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
   std::vector<int32_t> plan(static_cast<size_t>(heads * nb + n_rep * nbq_b));
   std::vector<uint8_t> active(static_cast<size_t>(heads));
   for (int c = 0; c < n_chunks; ++c) {
-    const int h0 = c * hpc, h1 = std::min(heads, h0 + hpc);
+    const int h0 = bound[c], h1 = bound[c + 1];
     std::vector<int32_t> rep_c;
     for (int h = 0; h < heads; ++h) active[h] = (h >= h0 && h < h1) ? 1 : 0;
     for (int i = 0; i < n_rep; ++i)
@@ -428,7 +438,8 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
   const size_t anchor_bytes =
       n_rep > 0 ? calibatt_repeat_workspace_size(std::min(hpc, n_rep), frames, H, W, k_anchor) : 0;
   uint8_t* ws8 = static_cast<uint8_t*>(ws);
-  int32_t* lists_dev = reinterpret_cast<int32_t*>(ws8 + ((anchor_bytes + 255) & ~static_cast<size_t>(255)));
+  const size_t anchor_stride = (anchor_bytes + 255) & ~static_cast<size_t>(255);
+  int32_t* lists_dev = reinterpret_cast<int32_t*>(ws8 + 2 * anchor_stride);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CALIBATT_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_pipe_mu[dev]);  // one caller of a device's pipe at a time
@@ -442,12 +453,14 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
       !ok(cudaMemcpyAsync(lists_dev, lists.data(), lists.size() * 4, cudaMemcpyHostToDevice, st)))
     return CALIBATT_ERR_CUDA;
   // the device buffers may still be in use by earlier work on the stream
-  if (!ok(cudaEventRecord(hp->ev[0], st)) || !ok(cudaStreamWaitEvent(hp->in, hp->ev[0], 0)))
+  if (!ok(cudaEventRecord(hp->ev[0], st)) || !ok(cudaStreamWaitEvent(hp->in, hp->ev[0], 0)) ||
+      !ok(cudaStreamWaitEvent(hp->cmp, hp->ev[0], 0)))
     return CALIBATT_ERR_CUDA;
   for (int c = 0; c < n_chunks; ++c) {
-    const int h0 = c * hpc, h1 = std::min(heads, h0 + hpc);
+    const int h0 = bound[c], h1 = bound[c + 1];
     const size_t off = static_cast<size_t>(h0) * head_elems, cnt = static_cast<size_t>(h1 - h0) * head_elems * 2;
     cudaEvent_t ev_in = hp->ev[2 + 2 * c], ev_done = hp->ev[3 + 2 * c];
+    cudaStream_t cs = (c & 1) ? hp->cmp : st;
     // q: runs of whole heads; a repeated head reads only its anchor pixel rows,
     // so only those are copied (one strided copy per anchor row: one W-token
     // row of every frame)
@@ -473,14 +486,15 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
     }
     if (!ok(cudaMemcpyAsync(k_dev + off, k_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
         !ok(cudaMemcpyAsync(v_dev + off, v_host + off, cnt, cudaMemcpyHostToDevice, hp->in)) ||
-        !ok(cudaEventRecord(ev_in, hp->in)) || !ok(cudaStreamWaitEvent(st, ev_in, 0)))
+        !ok(cudaEventRecord(ev_in, hp->in)) || !ok(cudaStreamWaitEvent(cs, ev_in, 0)))
       return CALIBATT_ERR_CUDA;
+    // chunks alternate between two compute streams and two anchor buffers
     rc = calibatt_mixed_attn_fwd(q_dev, k_dev, v_dev, heads, frames, H, W, d, k_anchor, scale, row_ptr, col_idx,
                                  nnz, n_rep_c[c] ? lists_dev + rep_off[c] : nullptr, n_rep_c[c],
-                                 n_work[c] ? lists_dev + work_off[c] : nullptr, n_work[c], o_dev, lse_dev, ws,
-                                 anchor_bytes, stream);
+                                 n_work[c] ? lists_dev + work_off[c] : nullptr, n_work[c], o_dev, lse_dev,
+                                 ws8 + (c & 1) * anchor_stride, anchor_bytes, reinterpret_cast<calibatt_stream_t>(cs));
     if (rc != CALIBATT_OK) return rc;
-    if (!ok(cudaEventRecord(ev_done, st)) || !ok(cudaStreamWaitEvent(hp->out, ev_done, 0)) ||
+    if (!ok(cudaEventRecord(ev_done, cs)) || !ok(cudaStreamWaitEvent(hp->out, ev_done, 0)) ||
         !ok(cudaMemcpyAsync(o_host + off, o_dev + off, cnt, cudaMemcpyDeviceToHost, hp->out)) ||
         (lse_host && !ok(cudaMemcpyAsync(lse_host + static_cast<size_t>(h0) * n, lse_dev + static_cast<size_t>(h0) * n,
                                          static_cast<size_t>(h1 - h0) * n * sizeof(float), cudaMemcpyDeviceToHost,

@@ -193,7 +193,11 @@ size_t calibatt_mixed_host_workspace_size(int heads, int frames, int H, int W, i
  * heads_per_chunk heads (<= 0: 2; on the Wan-720p workload 2 heads per chunk
  * measured best of 2, 3, 4, 5, 8 and 20): while the attention of chunk c runs on
  * `stream`, q, k, v of chunk c+1 are copied in on a second stream and o (and
- * lse) of chunk c-1 copied out on a third, so copies and compute overlap.
+ * lse) of chunk c-1 copied out on a third, so copies and compute overlap. The
+ * first chunk holds ceil(heads_per_chunk / 2) heads, so that the copy-in
+ * that nothing overlaps is short. Odd chunks run their attention on a fourth
+ * stream (with their own anchor buffer), so that a chunk's launch can start
+ * on the SMs that the previous chunk's last units leave idle.
  * Returns once everything is enqueued; the results are in o_host (lse_host)
  * when `stream` completes. Use page-locked host memory, else the copies do not
  * overlap. The skip list, work lists and repeated heads are those of
