@@ -307,7 +307,10 @@ def run_ours(args, world, rank, local):
     q, k, v = synth.qkv(wl, 1000 + rank, device=dev)
     row_ptr_h = row_ptr.cpu().numpy()
     head_active = np.array([h not in rep_heads for h in range(heads)], np.uint8)
-    work = torch.from_numpy(binding.build_plan(row_ptr_h, heads, nb, head_active)).to(dev)
+    # every work list is laid out for the device's worker slots (balanced
+    # static schedule; any order gives the same output)
+    work = torch.from_numpy(binding.balance_plan(binding.build_plan(row_ptr_h, heads, nb, head_active), row_ptr_h,
+                                                 heads, nb)).to(dev)
     rep_t = torch.tensor(rep_heads, dtype=torch.int32, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((heads, n), dtype=torch.float32, device=dev)
@@ -339,7 +342,7 @@ def run_ours(args, world, rank, local):
     else:
         work_np = binding.build_mixed_plan(row_ptr_h, heads, nb, rep_heads, wl.F, wl.H, wl.W, wl.k_anchor)
         my_rep, f_rank = rep_heads, f_step
-    work_mixed = torch.from_numpy(work_np).to(dev)
+    work_mixed = torch.from_numpy(binding.balance_plan(work_np, row_ptr_h, heads, nb)).to(dev)
     my_rep_t = torch.tensor(my_rep, dtype=torch.int32, device=dev)
 
     def step():
@@ -385,7 +388,9 @@ def run_ours(args, world, rank, local):
     # ---- 0 %-sparse run: the same kernel with every block kept, all 40 heads
     full = torch.ones((heads, nb, nb), dtype=torch.int16, device=dev).view(torch.uint16)
     _, rp_full, ci_full, _ = binding.aggregate_masks(full, 1, 0.5)
-    work_full = torch.from_numpy(binding.build_plan(rp_full.cpu().numpy(), heads, nb)).to(dev)
+    rp_full_h = rp_full.cpu().numpy()
+    work_full = torch.from_numpy(binding.balance_plan(binding.build_plan(rp_full_h, heads, nb), rp_full_h, heads,
+                                                      nb)).to(dev)
 
     def dense_call():
         binding.sparse_attn_fwd(q, k, v, rp_full, ci_full, work_full, o=o, lse=lse, stream=stream)

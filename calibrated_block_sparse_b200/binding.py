@@ -70,6 +70,7 @@ def load(build_if_missing: bool = False):
             "calibatt_aggregate_masks_noalloc": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P]),
             "calibatt_pixel_row_energy": (i32, [P, P, i32, i32, i32, i32, i32, f32, P, P, P, P]),
             "calibatt_build_mixed_plan": (i32, [P, i32, i32, P, i32, P, i32, i32, i32, i32, P, P]),
+            "calibatt_balance_plan": (i32, [P, i32, P, i32, i32, i32]),
             "calibatt_keep_histogram": (i32, [P, i32, i64, i32, P, P]),
             "calibatt_energy_workspace_size": (sz, [i32, i32]),
             "calibatt_shard_heads": (i32, [P, i32, i32, P, i32, i32, i32, i32, i32, P, P]),
@@ -171,6 +172,16 @@ def build_mixed_plan(row_ptr: np.ndarray, heads: int, nb: int, rep_heads, F: int
     _check(load().calibatt_build_mixed_plan(_ptr(rp), heads, nb, None, len(rep), _ptr(rep) if len(rep) else None,
                                             F, H, W, k_anchor, _ptr(out), _ptr(n)), "build_mixed_plan")
     return out[: int(n[0])].copy()
+
+
+def balance_plan(work_list: np.ndarray, row_ptr: np.ndarray, heads: int, nb: int, n_slots: int = 0) -> np.ndarray:
+    """calibatt_balance_plan on a copy of a host work list (n_slots <= 0: two
+    per SM of the current device)."""
+    w = np.array(work_list, dtype=np.int32, copy=True)
+    rp = np.ascontiguousarray(row_ptr, np.int32)
+    _check(load().calibatt_balance_plan(_ptr(w), int(w.size), _ptr(rp), int(heads), int(nb), int(n_slots)),
+           "calibatt_balance_plan")
+    return w
 
 
 def shard_heads(row_ptr: np.ndarray, heads: int, nb: int, rep_heads, F: int, W: int, k_anchor: int, n_ranks: int):

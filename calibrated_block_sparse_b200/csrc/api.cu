@@ -255,6 +255,47 @@ int calibatt_build_mixed_plan(const int32_t* row_ptr, int heads, int nb, const u
   return CALIBATT_OK;
 }
 
+int calibatt_balance_plan(int32_t* work_list, int32_t n_work, const int32_t* row_ptr, int heads, int nb,
+                          int n_slots) {
+  if (!work_list || n_work < 0 || !row_ptr || heads < 1 || nb < 1) return CALIBATT_ERR_ARG;
+  if (n_work == 0) return CALIBATT_OK;
+  if (n_slots <= 0) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      return CALIBATT_ERR_CUDA;
+    n_slots = 2 * sms;
+  }
+  if (n_slots < 2) return CALIBATT_ERR_ARG;
+  // the kernel's grid: one CTA of two slots per SM, no more CTAs than unit pairs
+  const int64_t ctas = std::min<int64_t>(n_slots / 2, (static_cast<int64_t>(n_work) + 1) / 2);
+  const int64_t G = 2 * ctas;
+  const int64_t n_a = static_cast<int64_t>(heads) * nb;
+  auto cost = [&](int32_t code) -> int64_t {
+    if (code >= 0 && code < n_a) return static_cast<int64_t>(row_ptr[code + 1]) - row_ptr[code] + 2;
+    if (code >= n_a) return nb + 2;  // anchor-query unit: every key block
+    return 2;
+  };
+  std::vector<int32_t> in(work_list, work_list + n_work);
+  std::vector<int64_t> load(static_cast<size_t>(G), 0);
+  std::vector<int64_t> units, slots;
+  for (int64_t r = 0; r * G < n_work; ++r) {
+    units.clear();
+    slots.clear();
+    for (int64_t i = r * G; i < std::min<int64_t>(n_work, (r + 1) * G); ++i) units.push_back(i);
+    auto pos = [&](int64_t g) { return r * G + ((r & 1) ? (G - 1 - g) : g); };
+    for (int64_t g = 0; g < G; ++g)
+      if (pos(g) < n_work) slots.push_back(g);
+    std::stable_sort(units.begin(), units.end(), [&](int64_t a, int64_t b) { return cost(in[a]) > cost(in[b]); });
+    std::stable_sort(slots.begin(), slots.end(), [&](int64_t a, int64_t b) { return load[a] < load[b]; });
+    for (size_t i = 0; i < units.size(); ++i) {
+      work_list[pos(slots[i])] = in[units[i]];
+      load[slots[i]] += cost(in[units[i]]);
+    }
+  }
+  return CALIBATT_OK;
+}
+
 int calibatt_shard_heads(const int32_t* row_ptr_host, int heads, int nb, const int32_t* rep_heads_host, int n_rep,
                          int frames, int W, int k_anchor, int n_ranks, int32_t* owner, int64_t* load) {
   if (!row_ptr_host || !owner || heads < 1 || nb < 1 || n_rep < 0 || n_rep > heads || (n_rep > 0 && !rep_heads_host) ||
@@ -427,6 +468,7 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
     int32_t nw = 0;
     rc = calibatt_build_mixed_plan(row_ptr_host, heads, nb, active.data(), static_cast<int>(rep_c.size()),
                                    rep_c.empty() ? nullptr : rep_c.data(), frames, H, W, k_anchor, plan.data(), &nw);
+    if (rc == CALIBATT_OK) rc = calibatt_balance_plan(plan.data(), nw, row_ptr_host, heads, nb, 0);
     if (rc != CALIBATT_OK) return rc;
     work_off[c] = static_cast<int>(lists.size());
     lists.insert(lists.end(), plan.begin(), plan.begin() + nw);

@@ -152,6 +152,7 @@ int calibatt_bank_put(calibatt_bank* bank, int t, int l, double eps, const int32
   int32_t n_work = 0;
   int rc = calibatt_build_mixed_plan(row_ptr_host, bank->heads, bank->nb, nullptr, n_rep, rep_heads_host,
                                      bank->frames, bank->H, bank->W, bank->k_anchor, work.data(), &n_work);
+  if (rc == CALIBATT_OK) rc = calibatt_balance_plan(work.data(), n_work, row_ptr_host, bank->heads, bank->nb, 0);
   if (rc != CALIBATT_OK) return rc;
   uint8_t* base = static_cast<uint8_t*>(dst);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -255,3 +255,52 @@ def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "library_path", lambda: str(tmp_path / "absent.so"))
     with pytest.raises(ImportError):
         b.load()
+
+
+def _slot_loads(work, cost, n_slots):
+    """Per-slot work under the kernels' static schedule: G = 2*min(n_slots/2,
+    ceil(n/2)) slots; slot g takes entry t*G + g in even rounds t and
+    t*G + G-1-g in odd ones."""
+    n = len(work)
+    G = 2 * min(n_slots // 2, (n + 1) // 2)
+    load = np.zeros(G, np.int64)
+    for i, code in enumerate(work):
+        t, q = divmod(i, G)
+        g = q if t % 2 == 0 else G - 1 - q
+        load[g] += cost[code]
+    return load, G
+
+
+@pytest.mark.parametrize("n_slots,seed", [(296, 1), (16, 2), (6, 3), (296, 4)])
+def test_balance_plan_permutes_within_rounds_and_evens_slot_loads(binding, n_slots, seed):
+    rng = np.random.default_rng(seed)
+    heads, nb = 7, 61
+    # heads of very different density, as calibrated masks give
+    kept = np.concatenate([rng.binomial(nb, p, nb) for p in rng.uniform(0.02, 0.9, heads)]).astype(np.int32)
+    row_ptr = np.concatenate([[0], np.cumsum(kept)]).astype(np.int32)
+    n_rep_units = 9  # anchor-query unit codes after the block-sparse ones
+    work = binding.build_plan(row_ptr, heads, nb)
+    work = np.concatenate([heads * nb + np.arange(n_rep_units, dtype=np.int32), work])
+    cost = np.concatenate([kept + 2, np.full(n_rep_units, nb + 2)])
+    out = binding.balance_plan(work, row_ptr, heads, nb, n_slots)
+    assert sorted(out.tolist()) == sorted(work.tolist())
+    load0, G = _slot_loads(work, cost, n_slots)
+    load1, _ = _slot_loads(out, cost, n_slots)
+    for r in range(0, len(work), G):  # every round keeps its own entries
+        assert sorted(out[r:r + G].tolist()) == sorted(work[r:r + G].tolist())
+    # matching the costliest unit of a round to the least-loaded slot keeps
+    # the spread within one unit's cost over the full rounds, two with the
+    # last, partial round
+    assert load1.max() - load1.min() <= 2 * cost.max()
+    assert load1.max() <= load0.max()
+    assert load1.sum() == load0.sum()
+
+
+def test_balance_plan_edge_cases(binding):
+    rp = np.array([0, 3, 3, 4], np.int32)
+    assert binding.balance_plan(np.zeros(0, np.int32), rp, 1, 3, 8).size == 0
+    w = np.array([2, 0, 1], np.int32)
+    assert sorted(binding.balance_plan(w, rp, 1, 3, 2).tolist()) == [0, 1, 2]  # one CTA: two slots
+    lib = binding.load()
+    assert lib.calibatt_balance_plan(binding._ptr(w), 3, binding._ptr(rp), 1, 3, 1) == -1  # fewer than 2 slots
+    assert lib.calibatt_balance_plan(None, 3, binding._ptr(rp), 1, 3, 8) == -1

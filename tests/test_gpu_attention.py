@@ -328,3 +328,33 @@ def test_mixed_launch_edge_cases(oracle):
     torch.cuda.synchronize()
     assert binding.get_status() == 0
     assert torch.equal(oh, o.cpu())
+
+
+def test_balanced_plan_gives_the_same_output():
+    """calibatt_balance_plan only reorders the work list: the mixed launch
+    writes bit for bit the same o and lse with the balanced list, laid out
+    for this device or for another slot count."""
+    binding = require_gpu()
+    F, H, W, heads, kk = 4, 8, 40, 6, 5
+    n = F * H * W
+    nb = (n + 127) // 128
+    q, k, v = synth.plain_qkv(heads, n, seed=123)
+    rng = np.random.default_rng(5)
+    mask = (rng.random((heads, nb, nb)) < rng.uniform(0.05, 0.95, (heads, 1, 1))).astype(np.uint8)
+    rp = np.concatenate([[0], np.cumsum(mask.reshape(-1, nb).sum(1))]).astype(np.int32)
+    ci = np.concatenate([np.nonzero(row)[0] for row in mask.reshape(-1, nb)]).astype(np.int32)
+    rep = [3]
+    dev = torch.device("cuda")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    rp_d, ci_d = torch.from_numpy(rp).to(dev), torch.from_numpy(ci).to(dev)
+    rep_d = torch.tensor(rep, dtype=torch.int32, device=dev)
+    w0 = binding.build_mixed_plan(rp, heads, nb, rep, F, H, W, kk)
+    outs = []
+    for w in (w0, binding.balance_plan(w0, rp, heads, nb), binding.balance_plan(w0, rp, heads, nb, 6)):
+        assert sorted(w.tolist()) == sorted(w0.tolist())
+        o, lse = binding.mixed_attn_fwd(qd, kd, vd, F, H, W, rp_d, ci_d, rep_d, torch.from_numpy(w).to(dev),
+                                        k_anchor=kk)
+        outs.append((o.cpu(), lse.cpu()))
+    assert binding.get_status() == 0
+    for o, lse in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(lse, outs[0][1])
