@@ -267,7 +267,7 @@ def graph_time(fn, reps, stream):
     return ms
 
 
-TRAFFIC_PER_TILE = 650.87e6 / 514058  # dram bytes per kept tile, measured (see the roofline block)
+TRAFFIC_PER_TILE = 565.24e6 / 514058  # dram bytes per kept tile, measured (see the roofline block)
 
 
 def run_ours(args, world, rank, local):
@@ -546,7 +546,7 @@ def run_ours(args, world, rank, local):
         kname += "; rank 0 share of the heads"
     # DRAM traffic per launch: the given figure, else the bytes per kept tile
     # of the one ncu capture (profiles/attn_kernel_wan720_5heads_ncu_full.md:
-    # 650.9 MB over 514 058 kept tiles) times the tiles of this launch
+    # 565.2 MB over 514 058 kept tiles) times the tiles of this launch
     mine = [h for h in sparse_heads if not shard or owner[h] == rank]
     tiles = int(sum(int(masks[h].sum()) for h in mine)) + len(my_rep) * -(-wl.F * wl.k_anchor * wl.W // 128) * nb
     traffic = args.traffic_bytes if args.traffic_bytes else TRAFFIC_PER_TILE * tiles
