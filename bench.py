@@ -401,6 +401,26 @@ def run_ours(args, world, rank, local):
     f_dense = float(4 * D * n * n * heads)
     del rp_full, ci_full, work_full, full
 
+    # ---- context, not this library's path: the same dense attention by the
+    # cuDNN backend of torch's scaled_dot_product_attention, timed the same way
+    library_dense = None
+    try:
+        import torch.nn.functional as F
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+
+        def library_call():
+            with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+                return F.scaled_dot_product_attention(q[None], k[None], v[None])
+
+        with torch.cuda.stream(stream):
+            library_call()
+            lib_ms = cuda_time(library_call, max(2, min(5, args.steps)), stream)
+        library_dense = {"kernel": "torch scaled_dot_product_attention, cuDNN backend, all blocks kept",
+                         "ms": lib_ms, "tflops": f_dense / (lib_ms * 1e-3) / 1e12,
+                         "step_speedup": lib_ms / ms_step}
+    except Exception as exc:  # the backend may be missing: report why
+        library_dense = {"unavailable": str(exc)[:200]}
+
     # ---- end to end through the C ABI with host buffers: H2D q,k,v, call, D2H o
     e2e = None
     if not args.no_e2e and not shard:
@@ -581,6 +601,7 @@ def run_ours(args, world, rank, local):
                                                   "sparse_tflops": f_sparse / (sparse_ms * 1e-3) / 1e12},
             "dense_ms": dense_ms, "dense_tflops": f_dense / (dense_ms * 1e-3) / 1e12,
             "speedup_vs_dense": dense_ms / ms_step,
+            "library_dense": library_dense,
             "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "calibration": calib,
             "clocks": clk.summary(),
         }
