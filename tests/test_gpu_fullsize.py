@@ -226,12 +226,44 @@ def test_wan720_mixed_launch_equals_separate_calls():
     rp_h = row_ptr.cpu().numpy()
     rep = list(wl.repeat_heads)
     rep_d = torch.tensor(rep, dtype=torch.int32, device=dev)
-    work = torch.from_numpy(binding.build_mixed_plan(rp_h, wl.heads, wl.nb, rep, wl.F, wl.H, wl.W)).to(dev)
+    # work lists laid out for this device, as the benchmark's are
+    work = torch.from_numpy(binding.balance_plan(
+        binding.build_mixed_plan(rp_h, wl.heads, wl.nb, rep, wl.F, wl.H, wl.W), rp_h, wl.heads, wl.nb)).to(dev)
     o, lse = binding.mixed_attn_fwd(q, k, v, wl.F, wl.H, wl.W, row_ptr, col_idx, rep_d, work)
     ha = np.array([h not in rep for h in range(wl.heads)], np.uint8)
-    work_s = torch.from_numpy(binding.build_plan(rp_h, wl.heads, wl.nb, ha)).to(dev)
+    work_s = torch.from_numpy(binding.balance_plan(binding.build_plan(rp_h, wl.heads, wl.nb, ha), rp_h, wl.heads,
+                                                   wl.nb)).to(dev)
     o2, lse2 = binding.sparse_attn_fwd(q, k, v, row_ptr, col_idx, work_s)
     binding.repeat_attn_fwd(q, k, v, wl.F, wl.H, wl.W, rep_d, o=o2, lse=lse2)
     assert binding.get_status() == 0
     assert torch.equal(o, o2)
     assert torch.equal(lse, lse2)
+
+
+def test_wan720_host_buffer_call_equals_device_call():
+    """The benchmark's end-to-end call (pinned host q, k, v in, o and lse out,
+    pipelined over chunks of 2 heads on two compute streams) returns bit for
+    bit the device call's o and lse at the full Wan-720p size."""
+    binding = require_gpu()
+    wl = synth.WORKLOADS["wan720"]
+    dev = torch.device(DEV)
+    q, k, v = synth.qkv(wl, 9, device=dev)
+    masks = synth.random_block_masks(wl)
+    row_ptr, col_idx = _skiplist(binding, masks, dev)
+    rp_h = row_ptr.cpu().numpy()
+    rep = list(wl.repeat_heads)
+    rep_d = torch.tensor(rep, dtype=torch.int32, device=dev)
+    work = torch.from_numpy(binding.build_mixed_plan(rp_h, wl.heads, wl.nb, rep, wl.F, wl.H, wl.W)).to(dev)
+    o_ref, lse_ref = binding.mixed_attn_fwd(q, k, v, wl.F, wl.H, wl.W, row_ptr, col_idx, rep_d, work)
+    o_ref, lse_ref = o_ref.cpu(), lse_ref.cpu()
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((wl.heads, wl.n), dtype=torch.float32).pin_memory()
+    bufs = [torch.empty_like(q) for _ in range(4)]
+    ld = torch.empty((wl.heads, wl.n), dtype=torch.float32, device=dev)
+    binding.mixed_attn_fwd_host(qh, kh, vh, oh, wl.F, wl.H, wl.W, rp_h, row_ptr, col_idx, rep, *bufs, lse_host=lh,
+                                lse_dev=ld, heads_per_chunk=2, k_anchor=wl.k_anchor)
+    torch.cuda.synchronize()
+    assert binding.get_status() == 0
+    assert torch.equal(oh, o_ref)
+    assert torch.equal(lh, lse_ref)
