@@ -2,9 +2,11 @@
 // repeated heads, on the sm_100a tensor core (explainer §三, online
 // inference): O = softmax(scale Q K^T) V over the kept 128 x 128 tiles.
 //
-// CTA (384 threads, one per SM, persistent over a longest-first unit list),
-// two independent query-tile "slots" so that the tensor core works on one
-// slot while the other slot's softmax runs:
+// CTA (384 threads, one per SM, persistent: slot g of G takes work-list
+// entries g, 2G-1-g, 2G+g, ..., which the host plan lays out head by head,
+// longest first, each round matched to the least-loaded slots), two
+// independent query-tile "slots" so that the tensor core works on one slot
+// while the other slot's softmax runs:
 //   warps 0-3  softmax warpgroup of slot 0 (thread = query row = TMEM lane)
 //   warps 4-7  softmax warpgroup of slot 1
 //   warp  8    TMA producer (one thread): Q tile per unit, K/V tiles per kept block
