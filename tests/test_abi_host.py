@@ -247,6 +247,16 @@ def test_workspace_sizes(binding):
     assert binding.repeat_workspace_size(8, 21, 45, 80, 5) == 8 * 21 * 5 * 80 * 256
     assert lib.calibatt_aggregate_workspace_size(40, 591) >= 40 * 591 * 4
     assert lib.calibatt_aggregate_workspace_size(0, 5) == 0
+    # host-buffer call: two anchor buffers (consecutive chunks may run at once)
+    # of min(heads per chunk, repeated heads) heads each, then every chunk's lists
+    nb = (21 * 45 * 80 + 127) // 128
+    anchors = binding.repeat_workspace_size(2, 21, 45, 80, 5)
+    lists = (40 * nb + 8 * (-(-21 * 5 * 80 // 128)) + 8) * 4
+    assert lib.calibatt_mixed_host_workspace_size(40, 21, 45, 80, 5, 8, 2) == 2 * anchors + (-(-lists // 256)) * 256
+    assert lib.calibatt_mixed_host_workspace_size(40, 21, 45, 80, 5, 8, 0) == \
+        lib.calibatt_mixed_host_workspace_size(40, 21, 45, 80, 5, 8, 2)
+    assert lib.calibatt_mixed_host_workspace_size(40, 21, 45, 80, 6, 8, 2) > 0
+    assert lib.calibatt_mixed_host_workspace_size(40, 21, 45, 80, 46, 8, 2) == 0  # k above H
 
 
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
