@@ -389,10 +389,12 @@ std::mutex g_pipe_mu[64];
 int host_pipe(int dev, int n_chunks, HostPipe** out) {
   static HostPipe pipes[64];
   HostPipe& hp = pipes[dev];
-  if (!hp.in && (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
-                 cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess ||
-                 cudaStreamCreateWithFlags(&hp.cmp, cudaStreamNonBlocking) != cudaSuccess))
-    return CALIBATT_ERR_CUDA;
+  // each stream on its own, so that a failed creation is retried on the next call
+  for (cudaStream_t* st : {&hp.in, &hp.out, &hp.cmp})
+    if (!*st && cudaStreamCreateWithFlags(st, cudaStreamNonBlocking) != cudaSuccess) {
+      *st = nullptr;
+      return CALIBATT_ERR_CUDA;
+    }
   while (static_cast<int>(hp.ev.size()) < 2 + 2 * n_chunks) {
     cudaEvent_t e;
     if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return CALIBATT_ERR_CUDA;
