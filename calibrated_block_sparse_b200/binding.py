@@ -54,6 +54,7 @@ def load(build_if_missing: bool = False):
             "calibatt_strerror": (ctypes.c_char_p, [i32]),
             "calibatt_version": (i32, []),
             "calibatt_get_status": (i32, [P]),
+            "calibatt_set_wait_limit": (i32, [f64]),
             "calibatt_eps_schedule": (f64, [f64, f64, f64, f64, f64]),
             "calibatt_validate_csr": (i32, [P, P, i32, i32, i64]),
             "calibatt_build_plan": (i32, [P, i32, i32, P, P, P]),
@@ -62,8 +63,8 @@ def load(build_if_missing: bool = False):
             "calibatt_sparse_attn_fwd": (i32, [P, P, P, i32, i32, i32, f32, P, P, i64, P, i32, P, P, P]),
             "calibatt_repeat_workspace_size": (sz, [i32, i32, i32, i32, i32]),
             "calibatt_repeat_attn_fwd": (i32, [P, P, P, i32, i32, i32, i32, i32, i32, f32, P, i32, P, P, P, sz, P]),
-            "calibatt_block_energy": (i32, [P, P, i32, i32, i32, f32, P, P, i32, f64, P, P, P, P]),
-            "calibatt_select_mask": (i32, [P, i32, i32, f64, P, P, P, P]),
+            "calibatt_block_energy": (i32, [P, P, i32, i32, i32, f32, P, P, i32, f64, P, P, P, P, f64, P]),
+            "calibatt_select_mask": (i32, [P, i32, i32, f64, P, P, P, P, f64, P]),
             "calibatt_accumulate_masks": (i32, [P, i64, P, P]),
             "calibatt_aggregate_workspace_size": (sz, [i32, i32]),
             "calibatt_aggregate_masks": (i32, [P, i32, i32, i32, f64, P, P, P, i64, P, P, sz, P]),
@@ -77,7 +78,8 @@ def load(build_if_missing: bool = False):
             "calibatt_mixed_host_workspace_size": (sz, [i32, i32, i32, i32, i32, i32, i32]),
             "calibatt_mixed_attn_fwd_host": (i32, [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, P, i64, P,
                                                    i32, i32, P, P, P, P, P, P, sz, P]),
-            "calibatt_block_energy_1pass": (i32, [P, P, i32, i32, i32, f32, P, sz, P, i32, f64, P, P, P, P, i32, P]),
+            "calibatt_block_energy_1pass": (i32, [P, P, i32, i32, i32, f32, P, sz, P, i32, f64, P, P, P, P, f64, P,
+                                                  i32, P]),
             "calibatt_bank_create": (P, [i32, i32, i32, i32, i32, i32, i32]),
             "calibatt_bank_destroy": (None, [P]),
             "calibatt_bank_entry_bytes": (sz, [P, i64, i32]),
@@ -139,6 +141,23 @@ def get_status(stream=None) -> int:
 
 def check_status(stream=None, what="kernel"):
     _check(get_status(stream), what)
+
+
+def set_wait_limit(seconds: float = 0.0):
+    """Limit of the bounded in-kernel waits of later launches on the current
+    device (0: the default of 2 s)."""
+    _check(load().calibatt_set_wait_limit(float(seconds)), "calibatt_set_wait_limit")
+
+
+TIE_WINDOW = 1e-6  # decisions within this distance of the threshold are counted
+
+
+def _tie_out(tie, rows_shape, dev):
+    if tie is True:
+        return torch.empty(rows_shape, dtype=torch.uint8, device=dev)
+    if tie is False or tie is None:
+        return None
+    return tie
 
 
 def eps_schedule(A, C, k, t, T) -> float:
@@ -328,10 +347,12 @@ def mixed_attn_fwd_host(q_host, k_host, v_host, o_host, F, H, W, row_ptr_host, r
 # ------------------------------------------------------------------ calibration
 
 def block_energy(q, k, eps=None, energy=True, mask=None, kept=None, counts=None, lse_ws=None, scale=None,
-                 stream=None):
-    """Block energy of one input; with eps, fused greedy selection too.
+                 stream=None, tie=None, tie_window=TIE_WINDOW):
+    """Block energy of one input; with eps, fused greedy selection too
+    (tie=True or a uint8 [heads][nb] tensor: tie-affected rows at tie_window).
 
-    Returns (energy or None, mask, kept, counts) — the outputs that were requested.
+    Returns (energy or None, mask, kept, counts) — the outputs that were
+    requested; with tie, (energy, mask, kept, counts, tie).
     """
     heads, n = _bhnd(q)
     nb = (n + BLOCK - 1) // BLOCK
@@ -347,12 +368,14 @@ def block_energy(q, k, eps=None, energy=True, mask=None, kept=None, counts=None,
     if fuse and mask is None and kept is None and counts is None:
         mask = torch.empty((heads, nb, nb), dtype=torch.uint8, device=dev)
         kept = torch.empty((heads, nb), dtype=torch.int32, device=dev)
+    want_tie = tie is not None and tie is not False
+    tie = _tie_out(tie, (heads, nb), dev)
     scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
     rc = load().calibatt_block_energy(_ptr(q), _ptr(k), heads, n, HEAD_DIM, scale, _ptr(lse_ws), _ptr(e),
                                       1 if fuse else 0, float(eps) if fuse else 0.0, _ptr(mask), _ptr(kept),
-                                      _ptr(counts), _stream(stream))
+                                      _ptr(counts), _ptr(tie), float(tie_window), _stream(stream))
     _check(rc, "calibatt_block_energy")
-    return e, mask, kept, counts
+    return (e, mask, kept, counts, tie) if want_tie else (e, mask, kept, counts)
 
 
 def pixel_row_energy(q, k, F, H, W, energy=False, pix=None, lse_ws=None, scale=None, stream=None):
@@ -403,10 +426,12 @@ def energy_workspace_size(heads: int, n: int) -> int:
 
 
 def block_energy_1pass(q, k, eps=None, energy=True, mask=None, kept=None, counts=None, pix=None, pix_W=None,
-                       ws=None, scale=None, stream=None):
+                       ws=None, scale=None, stream=None, tie=None, tie_window=TIE_WINDOW):
     """Block energy of one input in a single pass over the keys (with eps, the
     fused greedy selection too; with pix_W, pixel-row profiles of pix_W
-    consecutive queries). Returns (energy or None, mask, kept, counts, pix)."""
+    consecutive queries). Returns (energy or None, mask, kept, counts, pix);
+    with tie (True or a uint8 [heads][nb] tensor), (energy, mask, kept,
+    counts, pix, tie)."""
     heads, n = _bhnd(q)
     nb = (n + BLOCK - 1) // BLOCK
     dev = q.device
@@ -423,16 +448,20 @@ def block_energy_1pass(q, k, eps=None, energy=True, mask=None, kept=None, counts
         kept = torch.empty((heads, nb), dtype=torch.int32, device=dev)
     if pix_W is not None and pix is None:
         pix = torch.empty((heads, n // pix_W, nb), dtype=torch.float32, device=dev)
+    want_tie = tie is not None and tie is not False
+    tie = _tie_out(tie, (heads, nb), dev)
     scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
     rc = load().calibatt_block_energy_1pass(_ptr(q), _ptr(k), heads, n, HEAD_DIM, scale, _ptr(ws), ws.numel(),
                                             _ptr(e), 1 if fuse else 0, float(eps) if fuse else 0.0, _ptr(mask),
-                                            _ptr(kept), _ptr(counts), _ptr(pix), int(pix_W or 0), _stream(stream))
+                                            _ptr(kept), _ptr(counts), _ptr(tie), float(tie_window), _ptr(pix),
+                                            int(pix_W or 0), _stream(stream))
     _check(rc, "calibatt_block_energy_1pass")
-    return e, mask, kept, counts, pix
+    return (e, mask, kept, counts, pix, tie) if want_tie else (e, mask, kept, counts, pix)
 
 
-def select_mask(energy, eps, mask=True, kept=True, counts=None, stream=None):
-    """Greedy eps selection on [heads][nb][nb] energies; returns (mask, kept, counts)."""
+def select_mask(energy, eps, mask=True, kept=True, counts=None, stream=None, tie=None, tie_window=TIE_WINDOW):
+    """Greedy eps selection on [heads][nb][nb] energies; returns (mask, kept,
+    counts), and the tie-affected row flags when tie is True or a tensor."""
     _cuda_tensor(energy, torch.float32, "energy")
     heads, nb, _ = energy.shape
     dev = energy.device
@@ -444,10 +473,12 @@ def select_mask(energy, eps, mask=True, kept=True, counts=None, stream=None):
         kept = torch.empty((heads, nb), dtype=torch.int32, device=dev)
     elif kept is False:
         kept = None
+    want_tie = tie is not None and tie is not False
+    tie = _tie_out(tie, (heads, nb), dev)
     rc = load().calibatt_select_mask(_ptr(energy), heads, nb, float(eps), _ptr(mask), _ptr(kept), _ptr(counts),
-                                     _stream(stream))
+                                     _ptr(tie), float(tie_window), _stream(stream))
     _check(rc, "calibatt_select_mask")
-    return mask, kept, counts
+    return (mask, kept, counts, tie) if want_tie else (mask, kept, counts)
 
 
 def accumulate_masks(mask, counts, stream=None):

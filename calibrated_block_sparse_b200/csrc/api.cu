@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -32,6 +33,22 @@ int* status_word() {
     addr[dev] = static_cast<int*>(p);
   }
   return addr[dev];
+}
+
+// Limit of the bounded in-kernel waits per device (0: the default).
+std::atomic<uint64_t> g_wait_limit[64];
+
+uint64_t wait_limit_ns() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kWaitLimitNs;
+  const uint64_t v = g_wait_limit[dev].load(std::memory_order_relaxed);
+  return v ? v : kWaitLimitNs;
+}
+
+long long tie_window_fixed(double window) {
+  if (!(window > 0.0)) return 0;
+  if (window >= 8192.0) return LLONG_MAX;
+  return static_cast<long long>(std::llround(std::ldexp(window, 50)));
 }
 
 long long eps_to_fixed(double eps) {
@@ -66,6 +83,7 @@ KernelParams base_params() {
   KernelParams p;
   std::memset(&p, 0, sizeof p);
   p.status = status_word();
+  p.wait_limit_ns = wait_limit_ns();
   return p;
 }
 
@@ -120,7 +138,20 @@ const char* calibatt_strerror(int code) {
   }
 }
 
-int calibatt_version(void) { return 100; }
+int calibatt_version(void) { return 200; }
+
+int calibatt_set_wait_limit(double seconds) {
+  if (std::isnan(seconds) || seconds > 60.0) return CALIBATT_ERR_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CALIBATT_ERR_CUDA;
+  uint64_t ns = 0;  // default
+  if (seconds > 0.0) {
+    ns = static_cast<uint64_t>(std::llround(seconds * 1e9));
+    if (ns == 0) ns = 1;
+  }
+  g_wait_limit[dev].store(ns, std::memory_order_relaxed);
+  return CALIBATT_OK;
+}
 
 int calibatt_get_status(calibatt_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return CALIBATT_ERR_CUDA;
@@ -594,13 +625,13 @@ int calibatt_repeat_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, con
 
 int calibatt_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int n, int d, float scale,
                           float* lse_ws, float* energy, int fuse_select, double eps, uint8_t* mask, int32_t* kept,
-                          uint16_t* counts, calibatt_stream_t stream) {
+                          uint16_t* counts, uint8_t* tie, double tie_window, calibatt_stream_t stream) {
   int rc = check_qkv(q, k, nullptr, nullptr, heads, n, d);
   if (rc != CALIBATT_OK) return rc;
   const int nb = (n + 127) / 128;
   if (nb > CALIBATT_MAX_CALIB_NB) return CALIBATT_ERR_UNSUPPORTED;
-  if (!scale_ok(scale) || !lse_ws || std::isnan(eps)) return CALIBATT_ERR_ARG;
-  if (fuse_select && !mask && !kept && !counts) return CALIBATT_ERR_ARG;
+  if (!scale_ok(scale) || !lse_ws || std::isnan(eps) || std::isnan(tie_window)) return CALIBATT_ERR_ARG;
+  if (fuse_select && !mask && !kept && !counts && !tie) return CALIBATT_ERR_ARG;
   if (!aligned4(lse_ws) || (energy && !aligned4(energy)) || (kept && !aligned4(kept)) ||
       (counts && (reinterpret_cast<uintptr_t>(counts) & 1u)))
     return CALIBATT_ERR_ALIGN;
@@ -622,6 +653,8 @@ int calibatt_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int he
   p.mask = fuse_select ? mask : nullptr;
   p.kept = fuse_select ? kept : nullptr;
   p.counts = fuse_select ? counts : nullptr;
+  p.tie = fuse_select ? tie : nullptr;
+  p.tie_fx = tie_window_fixed(tie_window);
   return launch_attention(2, q, n, heads, k, nullptr, n, heads, p, st);
 }
 
@@ -636,15 +669,15 @@ size_t calibatt_energy_workspace_size(int heads, int n) {
 
 int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int n, int d,
                                 float scale, void* ws, size_t ws_bytes, float* energy, int fuse_select, double eps,
-                                uint8_t* mask, int32_t* kept, uint16_t* counts, float* pix_energy, int pix_W,
-                                calibatt_stream_t stream) {
+                                uint8_t* mask, int32_t* kept, uint16_t* counts, uint8_t* tie, double tie_window,
+                                float* pix_energy, int pix_W, calibatt_stream_t stream) {
   int rc = check_qkv(q, k, nullptr, nullptr, heads, n, d);
   if (rc != CALIBATT_OK) return rc;
   const int nb = (n + 127) / 128;
   if (nb > CALIBATT_MAX_CALIB_NB) return CALIBATT_ERR_UNSUPPORTED;
-  if (!scale_ok(scale) || !ws || std::isnan(eps)) return CALIBATT_ERR_ARG;
+  if (!scale_ok(scale) || !ws || std::isnan(eps) || std::isnan(tie_window)) return CALIBATT_ERR_ARG;
   if (ws_bytes < calibatt_energy_workspace_size(heads, n)) return CALIBATT_ERR_ARG;
-  if (fuse_select && !mask && !kept && !counts) return CALIBATT_ERR_ARG;
+  if (fuse_select && !mask && !kept && !counts && !tie) return CALIBATT_ERR_ARG;
   if (pix_energy && (pix_W < 1 || n % pix_W != 0)) return CALIBATT_ERR_ARG;
   if (!aligned16(ws) || (energy && !aligned4(energy)) || (kept && !aligned4(kept)) ||
       (counts && (reinterpret_cast<uintptr_t>(counts) & 1u)) || (pix_energy && !aligned4(pix_energy)))
@@ -664,6 +697,8 @@ int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, 
   p.mask = fuse_select ? mask : nullptr;
   p.kept = fuse_select ? kept : nullptr;
   p.counts = fuse_select ? counts : nullptr;
+  p.tie = fuse_select ? tie : nullptr;
+  p.tie_fx = tie_window_fixed(tie_window);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (pix_energy) {
     const size_t pix_bytes = static_cast<size_t>(heads) * (n / pix_W) * nb * sizeof(float);
@@ -677,14 +712,14 @@ int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, 
 }
 
 int calibatt_select_mask(const float* energy, int heads, int nb, double eps, uint8_t* mask, int32_t* kept,
-                         uint16_t* counts, calibatt_stream_t stream) {
-  if (!energy || heads < 1 || nb < 1 || std::isnan(eps)) return CALIBATT_ERR_ARG;
+                         uint16_t* counts, uint8_t* tie, double tie_window, calibatt_stream_t stream) {
+  if (!energy || heads < 1 || nb < 1 || std::isnan(eps) || std::isnan(tie_window)) return CALIBATT_ERR_ARG;
   if (nb > CALIBATT_MAX_CALIB_NB) return CALIBATT_ERR_UNSUPPORTED;
-  if (!mask && !kept && !counts) return CALIBATT_ERR_ARG;
+  if (!mask && !kept && !counts && !tie) return CALIBATT_ERR_ARG;
   if (!aligned4(energy) || (kept && !aligned4(kept)) || (counts && (reinterpret_cast<uintptr_t>(counts) & 1u)))
     return CALIBATT_ERR_ALIGN;
-  return launch_select(energy, static_cast<int64_t>(heads) * nb, nb, eps_to_fixed(eps), mask, kept, counts,
-                       reinterpret_cast<cudaStream_t>(stream));
+  return launch_select(energy, static_cast<int64_t>(heads) * nb, nb, eps_to_fixed(eps), mask, kept, counts, tie,
+                       tie_window_fixed(tie_window), reinterpret_cast<cudaStream_t>(stream));
 }
 
 int calibatt_accumulate_masks(const uint8_t* mask, int64_t cells, uint16_t* counts, calibatt_stream_t stream) {

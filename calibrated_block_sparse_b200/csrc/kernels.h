@@ -44,6 +44,8 @@ struct KernelParams {
   uint8_t* mask;
   int32_t* kept;
   uint16_t* counts;
+  uint8_t* tie;        // [heads_q][nbq] tie-affected flags of the fused selection, or NULL
+  long long tie_fx;    // tie window in fixed point (50 fraction bits)
   // pixel-row profiles (energy pass): pix_energy[hq][q / pix_W][c] += ... / pix_W
   float* pix_energy;   // [heads_q][pix_rows][nbk] or NULL
   int pix_W, pix_rows;
@@ -51,6 +53,7 @@ struct KernelParams {
   // single-pass energy: per slot, per key block, per row (tile sum, running max)
   float2* energy_ws;   // [2 * grid][nbk][128]
   int* status;         // device status word
+  uint64_t wait_limit_ns;  // limit of the pipeline's bounded waits
 };
 
 struct AnchorTable {
@@ -74,7 +77,7 @@ int launch_attention(int mode, const void* q, int q_rows, int q_heads, const voi
 long long eps_to_fixed(double eps);
 
 int launch_select(const float* energy, int64_t rows, int nb, long long eps_fx, uint8_t* mask, int32_t* kept,
-                  uint16_t* counts, cudaStream_t stream);
+                  uint16_t* counts, uint8_t* tie, long long tie_fx, cudaStream_t stream);
 int launch_accumulate(const uint8_t* mask, int64_t cells, uint16_t* counts, cudaStream_t stream);
 int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold, uint8_t* mask, int32_t* row_ptr,
                      int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* row_cnt, int* status,
@@ -86,5 +89,11 @@ int launch_gather(const void* q, int n, int heads, const int32_t* rep_heads, int
 
 // Device address of the status word on the current device (NULL on failure).
 int* status_word();
+
+// Limit of the bounded in-kernel waits of launches on the current device.
+uint64_t wait_limit_ns();
+
+// Tie window (in the greedy sum's units) in fixed point; 0 for none.
+long long tie_window_fixed(double window);
 
 }  // namespace calibatt

@@ -3,6 +3,9 @@
 // Every wait is bounded by a wall-clock limit read from %globaltimer; a wait
 // that runs out records CALIBATT_ERR_TIMEOUT in the device status word and
 // returns false so that the caller can wind down instead of hanging the GPU.
+// Pipeline waits take the launch's limit (calibatt_set_wait_limit); waits
+// that only drain work already issued (TMA copies, MMAs) keep the fixed
+// kWaitLimitNs, so that no CTA leaves with a copy or an MMA in flight.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -61,17 +64,49 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with an explicit suspend-time hint (nanoseconds): returns soon
+// after the hint when the phase is not complete.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t addr, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Limits below this are a test knob: such waits poll without suspending and
+// read the clock on every poll, so the first wait that is not already
+// complete runs out.
+constexpr uint64_t kShortWaitNs = 1000000ull;
+
 // Wait for the phase with the given parity to complete. Returns false (and
-// records a timeout) if it did not within kWaitLimitNs, or if *abort is set.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
+// records a timeout) if it did not within limit_ns, or if *abort is set.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t addr = smem_u32(bar);
+  if (limit_ns < kShortWaitNs) {
+    const uint64_t t0 = globaltimer();
+    while (true) {
+      if (mbar_try_wait_hint(addr, parity, 32u)) return true;
+      if (*abort) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        record_error(status, CALIBATT_ERR_TIMEOUT);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         record_error(status, CALIBATT_ERR_TIMEOUT);
         *abort = 1;
         return false;

@@ -196,6 +196,27 @@ inline int sm_count() {
   return n;
 }
 
+// One-time setup of a kernel per device. cudaFuncSetAttribute acts on the
+// current device, so a process that launches on several GPUs, or from several
+// host threads, needs it once for each device; the flags are per device and
+// read under a lock.
+struct PerDeviceOnce {
+  std::mutex mu;
+  bool done[64] = {};
+};
+
+inline int set_max_smem_once(const void* fn, int bytes, PerDeviceOnce& once) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CALIBATT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(once.mu);
+  if (!once.done[dev]) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+      return CALIBATT_ERR_CUDA;
+    once.done[dev] = true;
+  }
+  return CALIBATT_OK;
+}
+
 // Energy-pass launcher (score.cu) and the grid it uses for n_units work units
 // (one CTA of two slots per SM at most).
 int launch_score(int mode, const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams& p, cudaStream_t stream);

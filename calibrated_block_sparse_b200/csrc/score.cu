@@ -124,14 +124,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         Cursor& c = cur[s];
         if (!c.valid) continue;
         if (c.j == 0) {
-          if (!(ok = mbar_wait(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status))) break;
+          if (!(ok = mbar_wait(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns))) break;
           uint8_t* dst = smem + L::kQOff + s * kTile;
           mbar_arrive_expect_tx(&bar.q_full[s], kTile);
           tma_load_3d(dst, &tm_q, &bar.q_full[s], 0, c.u.r * 128, c.u.hq);
           tma_load_3d(dst + kHalf, &tm_q, &bar.q_full[s], 64, c.u.r * 128, c.u.hq);
           ++n_q[s];
         }
-        if (!(ok = mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns))) break;
         bar.first[stage] = c.j == 0;
         bar.last[stage] = c.j == c.u.nnz - 1;
         bar.slot[stage] = s;
@@ -146,14 +146,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         cursor_next(p, 2 * blockIdx.x + s, G, c);
       }
     }
-    if (ok && mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status)) {
+    bool marker = false;
+    if (ok && mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
       bar.end = 1;
       bar.slot[stage] = 2;  // end marker
       mbar_arrive(&bar.ring_full[stage]);
+      marker = true;
     }
-    // no copy may still be landing when the CTA leaves
+    // no copy may still be landing when the CTA leaves: wait for the latest
+    // phase of every ring stage and Q buffer. With the end marker sent, the
+    // latest phase of `stage` is the marker's own (its earlier copy was
+    // consumed before the producer could reuse the stage); without it (a
+    // wait failed), `stage` was not armed again and its latest phase is the
+    // previous lap's.
     for (int i = 0; i < kScoreRing; ++i) {
-      int st = static_cast<int>(stage) - i;
+      int st = static_cast<int>(stage) - (marker ? 0 : 1) - i;
       uint32_t ph = phase;
       if (st < 0) {
         st += kScoreRing;
@@ -173,7 +180,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const uint64_t qdesc0 = desc_k_base(sbase + L::kQOff);
     const uint64_t kdesc0 = desc_k_base(sbase + L::kRingOff);
     while (true) {
-      if (!mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status)) break;
+      if (!mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status, p.wait_limit_ns)) break;
       // read every word of the stage now: once ring_empty is committed below,
       // the producer may reuse the stage and rewrite them for its next tile
       const uint32_t s = *reinterpret_cast<volatile uint32_t*>(&bar.slot[stage]);
@@ -181,10 +188,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       const bool first = *reinterpret_cast<volatile uint32_t*>(&bar.first[stage]) != 0;
       const bool last = *reinterpret_cast<volatile uint32_t*>(&bar.last[stage]) != 0;
       if (first) {
-        if (!mbar_wait(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status)) break;
+        if (!mbar_wait(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status, p.wait_limit_ns)) break;
       }
       const int buf = n_s[s] & 1;
-      if (!mbar_wait(&bar.s_empty[s][buf], ((n_s[s] >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+      if (!mbar_wait(&bar.s_empty[s][buf], ((n_s[s] >> 1) & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + (2 * s + buf) * 128;
       const uint64_t qd = qdesc0 + s * (kTile >> 4), kd = kdesc0 + stage * (kTile >> 4);
@@ -256,7 +263,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const int buf = n_sfull & 1;
         float acc = 0.f;
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_full[s][buf], (n_sfull >> 1) & 1, abort_flag,
-                                                       p.status));
+                                                       p.status, p.wait_limit_ns));
         if (ok) {
           ++n_sfull;
           tc_fence_after();
@@ -357,11 +364,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           if (p.energy && ok) p.energy[erow + c] = e;
         }
         if (p.fuse_select) {
+          // the finished row is selected by the warpgroup's first warp
+          // (its 8 KB histogram behind the row in the slot's scratch)
           named_bar_sync(1 + s, 128);
-          SelectOut out{p.mask ? p.mask + erow : nullptr, p.kept ? p.kept + (erow / p.nbk) : nullptr,
-                        p.counts ? p.counts + erow : nullptr};
-          if (!ok) out = SelectOut{nullptr, nullptr, nullptr};
-          select_row<8>(part, p.nbk, p.eps_fx, reinterpret_cast<uint8_t*>(part + 1024), row, 128, 1 + s, out);
+          if (wl == 0) {
+            const int64_t urow = erow / p.nbk;
+            SelectOut out{p.mask ? p.mask + erow : nullptr, p.kept ? p.kept + urow : nullptr,
+                          p.counts ? p.counts + erow : nullptr, p.tie ? p.tie + urow : nullptr};
+            if (!ok) out = SelectOut{nullptr, nullptr, nullptr, nullptr};
+            warp_select<32>(part, p.nbk, p.eps_fx, p.tie_fx, reinterpret_cast<unsigned long long*>(part + 1024), out);
+          }
         }
         named_bar_sync(1 + s, 128);
       }
@@ -382,13 +394,10 @@ template <int MODE>
 int launch_mode(const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams& p, cudaStream_t stream) {
   using L = ScoreLayout<MODE>;
   static_assert(L::kDynSmem <= 232448, "shared memory budget");
-  static bool configured = false;  // per process; the attribute is per function
-  if (!configured) {
-    if (cudaFuncSetAttribute(score_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
-        cudaSuccess)
-      return CALIBATT_ERR_CUDA;
-    configured = true;
-  }
+  static_assert(kEnergyScratch >= 4096 + kSelectScratchBytes, "selection scratch behind the energy row");
+  static PerDeviceOnce smem_once;
+  const int rc = set_max_smem_once(reinterpret_cast<const void*>(score_kernel<MODE>), L::kDynSmem, smem_once);
+  if (rc != CALIBATT_OK) return rc;
   if (p.n_units <= 0) return CALIBATT_OK;
   score_kernel<MODE><<<score_grid(p.n_units), kScoreThreads, L::kDynSmem, stream>>>(mq, mk, p);
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;

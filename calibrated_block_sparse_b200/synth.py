@@ -96,8 +96,27 @@ def head_sigma(wl: Workload, head: int) -> float:
     return float(math.exp(math.log(lo) + u * (math.log(hi) - math.log(lo))))
 
 
-def fourier_features(wl: Workload, head: int) -> torch.Tensor:
-    """e(pos) for every token of one head, zero-padded to d: [n, 128] float32."""
+_FEATURE_CACHE = {}
+
+
+def fourier_features(wl: Workload, head: int, device="cpu") -> torch.Tensor:
+    """e(pos) for every token of one head, zero-padded to d: [n, 128] float32.
+
+    The features depend on the head only (not on the input), so they are
+    computed once per (workload, head, device) and kept."""
+    key = (wl, head, str(device))
+    hit = _FEATURE_CACHE.get(key)
+    if hit is None:
+        hit = _fourier_features(wl, head).to(device)
+        _FEATURE_CACHE[key] = hit
+    return hit
+
+
+def clear_feature_cache():
+    _FEATURE_CACHE.clear()
+
+
+def _fourier_features(wl: Workload, head: int) -> torch.Tensor:
     rng = np.random.default_rng(_seed(wl.config_id, 11, head))
     sigma = head_sigma(wl, head)
     w = rng.normal(0.0, sigma, size=(N_FEAT, 3))
@@ -126,7 +145,7 @@ def qkv(wl: Workload, input_idx: int, heads=None, with_v: bool = True, device="c
     heads = list(range(wl.heads)) if heads is None else list(heads)
     qs, ks, vs = [], [], []
     for h in heads:
-        e = fourier_features(wl, h).to(device)
+        e = fourier_features(wl, h, device)
         qs.append((_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 1), device) + 2.0 * e).to(torch.bfloat16))
         ks.append((_normal((wl.n, D_HEAD), _seed(wl.config_id, input_idx, h, 2), device) + 2.0 * e).to(torch.bfloat16))
         if with_v:

@@ -64,9 +64,24 @@ const char* calibatt_strerror(int code);
 /* Library ABI version (major*100 + minor). */
 int calibatt_version(void);
 
-/* Synchronises `stream`, then returns and clears the device status word
- * (CALIBATT_OK if no kernel recorded a fault since the last call). */
+/* Synchronises `stream`, then returns and clears the status word of the
+ * current device (CALIBATT_OK if no kernel recorded a fault since the last
+ * call). There is one word per device, not per stream: a fault recorded by a
+ * kernel on any stream of the device is reported (and cleared) here, and when
+ * several kernels fault only the first code is kept. Callers that need to
+ * tell streams apart serialise their status checks. */
 int calibatt_get_status(calibatt_stream_t stream);
+
+/* Limit, in seconds, of every bounded in-kernel wait of the launches made
+ * later on the current device (default 2 s; seconds <= 0 restores it; at most
+ * 60). A pipeline wait that runs out makes the kernel wind down without
+ * touching its outputs further and record CALIBATT_ERR_TIMEOUT for
+ * calibatt_get_status; the GPU context stays usable. Waits that only drain
+ * copies and tensor-core work already issued keep the default limit, so no
+ * kernel exits with work in flight. A short limit is a test knob: it makes the
+ * first wait that is not already satisfied run out.
+ * Returns CALIBATT_ERR_ARG for NaN or > 60 s. */
+int calibatt_set_wait_limit(double seconds);
 
 /* ---------------------------------------------------------------- host helpers */
 
@@ -251,15 +266,17 @@ int calibatt_mixed_attn_fwd_host(const calibatt_bf16* q_host, const calibatt_bf1
  * tile by tile.
  * When fuse_select != 0 the same kernel applies the greedy selection of
  * calibatt_select_mask at `eps` to each finished energy row and writes mask
- * and/or kept and/or adds the mask into counts.
+ * and/or kept and/or tie and/or adds the mask into counts.
  *   lse_ws : device fp32 scratch [heads][nb*128]
  *   energy : device fp32 [heads][nb][nb] or NULL
  *   mask   : device uint8 [heads][nb][nb] or NULL; kept: device int32 [heads][nb] or NULL
  *   counts : device uint16 [heads][nb][nb] or NULL (counts += mask)
+ *   tie, tie_window : as in calibatt_select_mask
  * Requires nb <= CALIBATT_MAX_CALIB_NB. */
 int calibatt_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int n, int d, float scale,
                           float* lse_ws, float* energy, int fuse_select, double eps, uint8_t* mask,
-                          int32_t* kept, uint16_t* counts, calibatt_stream_t stream);
+                          int32_t* kept, uint16_t* counts, uint8_t* tie, double tie_window,
+                          calibatt_stream_t stream);
 
 /* Workspace bytes of calibatt_block_energy_1pass for heads x n tokens on the
  * current device (it depends on the number of SMs; 0 on bad sizes). */
@@ -279,8 +296,8 @@ size_t calibatt_energy_workspace_size(int heads, int n);
  * Other arguments and outputs as in calibatt_block_energy. */
 int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int n, int d,
                                 float scale, void* ws, size_t ws_bytes, float* energy, int fuse_select, double eps,
-                                uint8_t* mask, int32_t* kept, uint16_t* counts, float* pix_energy, int pix_W,
-                                calibatt_stream_t stream);
+                                uint8_t* mask, int32_t* kept, uint16_t* counts, uint8_t* tie, double tie_window,
+                                float* pix_energy, int pix_W, calibatt_stream_t stream);
 
 /* Greedy eps selection (explainer §三, step 3) on rows of block energies:
  * order the row's blocks by energy descending (equal energies: lower column
@@ -292,9 +309,17 @@ int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, 
  *   energy : device fp32 [rows][nb], rows = heads*nb
  *   mask   : device uint8 [rows][nb] or NULL; kept: device int32 [rows] or NULL
  *   counts : device uint16 [rows][nb] or NULL (counts += mask)
+ *   tie    : device uint8 [rows] or NULL: 1 where the row's decision is
+ *            tie-affected at tie_window: the running sum with or without the
+ *            last kept block (in greedy order) lies within tie_window of eps,
+ *            or the last kept block's energy exceeds the next block's by less
+ *            than tie_window (the next block in greedy order; none when every
+ *            block is kept). Such decisions can flip under a perturbation of
+ *            the energies of that size; the benchmark counts them at 1e-6.
+ *   tie_window : >= 0 (0: no row is flagged); ignored when tie is NULL
  * Requires nb <= CALIBATT_MAX_CALIB_NB. */
 int calibatt_select_mask(const float* energy, int heads, int nb, double eps, uint8_t* mask, int32_t* kept,
-                         uint16_t* counts, calibatt_stream_t stream);
+                         uint16_t* counts, uint8_t* tie, double tie_window, calibatt_stream_t stream);
 
 /* counts[i] += mask[i] (saturating at 65535) for `cells` entries: folds one
  * calibration input's mask into the running sum over inputs (explainer §三). */

@@ -38,3 +38,54 @@ def compare_masks(mask_gpu, mask_ref, affected):
     diff = np.any(mg != mr, axis=1)
     aff = affected.reshape(-1)
     return int(diff.sum()), int(aff.sum()), int((diff & ~aff).sum())
+
+
+# ---------------------------------------------------------------- energy tolerance and tie windows
+#
+# Energies computed on the GPU (fp32 scores from the tensor core, an fp32
+# log-sum-exp, ex2.approx, fp32 tile sums) are accepted against the fp64
+# oracle at |E - E_ref| <= ENERGY_REL * E_ref + ENERGY_ABS * max_c E_ref[r, c]
+# per entry: the relative tolerance of 1e-5 on row entries that the parity
+# contract fixes (the rounding of the scores, the log-sum-exp, ex2.approx and
+# the tile sums adds up to a few 1e-6 relative; measured worst 1.9e-6), plus a
+# floor for the probabilities below 2^-126 that ex2.approx.ftz flushes to zero.
+ENERGY_REL = 1e-5
+ENERGY_ABS = 1e-12
+NORTH_STAR_TIE = 1e-6  # the tie window when both sides select from the same energies
+
+
+def energy_bound(E_ref):
+    return ENERGY_REL * E_ref + ENERGY_ABS * E_ref.max(-1, keepdims=True)
+
+
+def energy_ok(E, E_ref):
+    """(all entries within the bound, worst |E - E_ref| / bound, worst relative error)."""
+    b = energy_bound(E_ref)
+    d = np.abs(E - E_ref)
+    rel = d / np.maximum(E_ref, 1e-300)
+    return bool(np.all(d <= b)), float(np.max(d / np.maximum(b, 1e-300))), float(np.max(np.where(E_ref > 0, rel, 0)))
+
+
+def independent_tie_window(E_ref):
+    """Per-row window for comparing a selection made from GPU energies with one
+    made from the oracle's energies of the same input. Within the accepted
+    energy bound every running sum of the greedy order moves by at most the sum
+    of the per-entry bounds, and two energies can swap order only when they are
+    closer than their two bounds: so a row whose cut lies within
+    sum_c bound_c (plus the 1e-6 spec window) of eps, or whose energies
+    at the cut are that close, may legitimately differ. Shape: rows."""
+    return energy_bound(E_ref).sum(-1) + NORTH_STAR_TIE
+
+
+def cells_explained(agg_gpu, agg_ref, affected_rows):
+    """Per-cell attribution of aggregated-mask differences.
+
+    agg_gpu, agg_ref: [heads][nb][nb] aggregated masks; affected_rows:
+    [n_inputs][heads][nb] booleans, the (input, head, block-row) selections
+    that are tie-affected. A cell (h, r, c) may differ only if at least one
+    input's selection of row (h, r) is tie-affected; returns (n_diff_cells,
+    n_unexplained_cells)."""
+    diff = agg_gpu != agg_ref
+    row_aff = np.any(affected_rows, axis=0)  # [heads][nb]
+    unexplained = diff & ~row_aff[..., None]
+    return int(diff.sum()), int(unexplained.sum())

@@ -133,10 +133,18 @@ def test_argument_errors_are_caught_on_the_host(binding):
                                         1 << 30, None) == -4
     # calibration beyond 1024 blocks per row
     assert lib.calibatt_block_energy(fake, fake, 1, 1025 * 128, 128, 0.1, fake, None, 0, 0.0, None, None, None,
-                                     None) == -4
-    assert lib.calibatt_select_mask(fake, 1, 2000, 0.9, fake, None, None, None) == -4
-    assert lib.calibatt_select_mask(fake, 1, 16, 0.9, None, None, None, None) == -1
-    assert lib.calibatt_select_mask(fake, 1, 16, float("nan"), fake, None, None, None) == -1
+                                     None, 0.0, None) == -4
+    assert lib.calibatt_block_energy(fake, fake, 1, 1024, 128, 0.1, fake, None, 1, 0.9, None, None, None,
+                                     None, 0.0, None) == -1  # fused selection with no output
+    assert lib.calibatt_block_energy(fake, fake, 1, 1024, 128, 0.1, fake, None, 1, 0.9, None, None, None,
+                                     fake, float("nan"), None) == -1
+    assert lib.calibatt_select_mask(fake, 1, 2000, 0.9, fake, None, None, None, 0.0, None) == -4
+    assert lib.calibatt_select_mask(fake, 1, 16, 0.9, None, None, None, None, 0.0, None) == -1
+    assert lib.calibatt_select_mask(fake, 1, 16, float("nan"), fake, None, None, None, 0.0, None) == -1
+    assert lib.calibatt_select_mask(fake, 1, 16, 0.9, None, None, None, fake, float("nan"), None) == -1
+    # the wait limit: NaN and more than a minute are refused before any device call
+    assert lib.calibatt_set_wait_limit(float("nan")) == -1
+    assert lib.calibatt_set_wait_limit(61.0) == -1
     # aggregation: short workspace, zero inputs
     assert lib.calibatt_aggregate_masks(fake, 4, 1, 16, 0.5, fake, fake, fake, 256, fake, fake, 4, None) == -1
     assert lib.calibatt_aggregate_masks(fake, 0, 1, 16, 0.5, fake, fake, fake, 256, fake, fake, 1024, None) == -1
@@ -201,9 +209,9 @@ def test_bank_index_on_the_host(binding):
         lib.calibatt_bank_destroy(b)
     # single-pass energy: short workspace, pixel rows that do not divide n
     assert lib.calibatt_block_energy_1pass(P(0x100000), P(0x100000), 1, 4096, 128, 0.1, P(0x100000), 16, None, 0,
-                                           0.0, None, None, None, None, 0, None) == -1
+                                           0.0, None, None, None, None, 0.0, None, 0, None) == -1
     assert lib.calibatt_block_energy_1pass(P(0x100000), P(0x100000), 1, 4096, 128, 0.1, P(0x100000), 1 << 40,
-                                           None, 0, 0.0, None, None, None, P(0x100000), 100, None) == -1
+                                           None, 0, 0.0, None, None, None, None, 0.0, P(0x100000), 100, None) == -1
     # host-buffer pipeline: short workspace, missing host buffer
     assert lib.calibatt_mixed_attn_fwd_host(fake, fake, fake, fake, None, 2, 2, 8, 16, 128, 5, 0.1, fake, fake, fake,
                                             4, None, 0, 8, fake, fake, fake, fake, None, fake, 4, None) == -1

@@ -1,8 +1,9 @@
 """The allocation-free skip-list build (calibatt_aggregate_masks_noalloc),
 for callers that cannot allocate device memory themselves: it must give the
 same mask, row_ptr, col_idx and nnz as calibatt_aggregate_masks with a
-caller-supplied workspace (integer work: bit-exact), on two calls in a row
-that share its static scratch array.
+caller-supplied workspace and as the oracle's binarisation and skip list
+(integer work: bit-exact), on two calls in a row that share its static
+scratch array.
 
 Named so that pytest collects it last; it passes alone in a fresh process too.
 """
@@ -23,7 +24,7 @@ def _outputs(heads, nb, dev):
 
 
 @pytest.mark.parametrize("heads,nb,n_inputs,rho", [(40, 591, 16, 0.5), (3, 37, 8, 0.3)])
-def test_noalloc_matches_workspace_variant_twice(heads, nb, n_inputs, rho):
+def test_noalloc_matches_workspace_variant_twice(oracle, heads, nb, n_inputs, rho):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from calibrated_block_sparse_b200 import binding
@@ -50,6 +51,13 @@ def test_noalloc_matches_workspace_variant_twice(heads, nb, n_inputs, rho):
         assert torch.equal(mask, ref[0])
         assert torch.equal(row_ptr, ref[1])
         assert torch.equal(col_idx[:total], ref[2][:total])
+        # and the oracle's rule written out: keep where count / n >= rho
+        m_ref = oracle.binarize_counts(counts_h.astype(np.int32), n_inputs, rho)
+        rp_ref, ci_ref = oracle.mask_to_csr(m_ref)
+        np.testing.assert_array_equal(mask.cpu().numpy(), m_ref)
+        np.testing.assert_array_equal(row_ptr.cpu().numpy(), rp_ref)
+        np.testing.assert_array_equal(col_idx[:total].cpu().numpy(), ci_ref)
+        assert total == ci_ref.size
 
 
 def test_noalloc_rejects_oversize():
