@@ -73,6 +73,11 @@ def _load():
             lib.oracle_pixel_row_energy.restype = None
             lib.oracle_spatial_score.argtypes = [P, i32, i32, i64, i32]
             lib.oracle_spatial_score.restype = f64
+            lib.oracle_anchor_block_energy.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, f64, P, i64, P, i32]
+            lib.oracle_anchor_block_energy.restype = ctypes.c_int
+            lib.oracle_repeat_attention_masked.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, f64, P, P,
+                                                           i64, P, P, i32]
+            lib.oracle_repeat_attention_masked.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -296,3 +301,61 @@ def keep_histogram(counts, n_inputs):
     if c.size and (c.min() < 0 or c.max() > n_inputs):
         raise ValueError("a count lies outside [0, n_inputs]")
     return np.stack([np.bincount(row, minlength=n_inputs + 1) for row in c]).astype(np.int64)
+
+
+def anchor_blocks(F, H, W, k_anchor, B=128):
+    """Number of blocks of B packed anchor queries of one repeated head."""
+    return (F * k_anchor * W + B - 1) // B
+
+
+def anchor_block_energy(q, k, F, H, W, k_anchor=5, B=128, scale=None, blockrows=None, threads=None):
+    """Block energy of the anchor queries of a repeated head (explainer §三:
+    calibration per (t, l, h); the same energy as block_energy, over the
+    head's anchor queries taken in the order frame, anchor, column and grouped
+    into blocks of B). Returns [h][nbq][nb] (or [len(blockrows)][nb] for
+    blockrows h*nbq + r)."""
+    q, k = _bf16_bits(q), _bf16_bits(k)
+    h, n, d = q.shape
+    assert n == F * H * W
+    nb = (n + B - 1) // B
+    nbq = anchor_blocks(F, H, W, k_anchor, B)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    if blockrows is None:
+        br, nbr = None, h * nbq
+    else:
+        br = np.ascontiguousarray(blockrows, dtype=np.int64)
+        nbr = br.size
+    E = np.empty((nbr, nb), np.float64)
+    rc = _load().oracle_anchor_block_energy(_ptr(q), _ptr(k), h, F, H, W, d, B, k_anchor, scale, _ptr(br), nbr,
+                                            _ptr(E), _threads(threads))
+    if rc != 0:
+        raise ValueError("k_anchor must be in [1, H]")
+    return E.reshape(h, nbq, nb) if blockrows is None else E
+
+
+def repeat_attention_masked(q, k, v, F, H, W, mask_b, k_anchor=5, B=128, scale=None, rows=None, threads=None):
+    """Repeated head whose anchor queries attend only to the key blocks their
+    anchor block's mask keeps (mask_b [h][nbq][nb]); every row copies its
+    nearest anchor row's output (explainer §三 and §六)."""
+    q, k, v = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    h, n, d = q.shape
+    assert n == F * H * W
+    nb = (n + B - 1) // B
+    nbq = anchor_blocks(F, H, W, k_anchor, B)
+    mask_b = np.ascontiguousarray(mask_b, dtype=np.uint8)
+    assert mask_b.shape == (h, nbq, nb)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    if rows is None:
+        o = np.empty((h, n, d), np.float64)
+        lse = np.empty((h, n), np.float64)
+        nr, rp = h * n, None
+    else:
+        rp = np.ascontiguousarray(rows, dtype=np.int64)
+        nr = rp.size
+        o = np.empty((nr, d), np.float64)
+        lse = np.empty((nr,), np.float64)
+    rc = _load().oracle_repeat_attention_masked(_ptr(q), _ptr(k), _ptr(v), h, F, H, W, d, B, k_anchor, scale,
+                                                _ptr(mask_b), _ptr(rp), nr, _ptr(o), _ptr(lse), _threads(threads))
+    if rc != 0:
+        raise ValueError("k_anchor must be in [1, H]")
+    return o, lse

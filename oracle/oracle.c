@@ -473,3 +473,151 @@ double oracle_spatial_score(const double *Epx, int F, int H, int64_t nb, int k_a
     free(owner);
     return count ? total / (double)count : 1.0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* 8. Repeated heads with a block mask on their anchor rows (explainer §三:  */
+/*    the two run-time decisions, a skip list for a head's blocks and the    */
+/*    spatial repetition of its rows, are both made per (t, l, h); the pages */
+/*    do not combine them, and this reading applies both: a repeated head    */
+/*    computes only its anchor rows, and those anchor queries attend only to */
+/*    the key blocks their own calibrated mask keeps).                       */
+/*    The anchor queries of a head are taken in the order frame, anchor,     */
+/*    column: packed row a = f*k*W + j*W + c is token f*H*W + a_j*W + c.     */
+/*    They are grouped into blocks of B packed rows (the last one ragged),   */
+/*    and calibrated exactly like query blocks: the energy of packed block   */
+/*    r over key block c is (1/|I_r|) sum_{i in I_r, j in J_c} P_ij.         */
+/*    At run time the anchor query in packed block r attends to the keys of  */
+/*    the kept blocks mask_b[h][r][*], and every row takes the output of its */
+/*    nearest anchor row (same frame, same column), as in section 2.         */
+/* ------------------------------------------------------------------------ */
+static int64_t packed_to_token(int64_t a, int W, int H, int k_anchor, const int *anchors) {
+    int64_t kw = (int64_t)k_anchor * W;
+    int64_t f = a / kw, rem = a % kw;
+    int64_t j = rem / W, c = rem % W;
+    return f * (int64_t)H * W + (int64_t)anchors[j] * W + c;
+}
+
+typedef struct {
+    const uint16_t *q, *k;
+    int d, B, H, W, k_anchor;
+    int64_t n, nq, nbq, nb; /* nq = F*k*W packed anchor queries per head */
+    double scale;
+    const int *anchors;
+    const int64_t *blockrows;
+    double *E;
+} anchor_energy_ctx;
+
+static void anchor_energy_blockrow(void *vctx, int64_t idx, double *s) {
+    anchor_energy_ctx *c = (anchor_energy_ctx *)vctx;
+    int64_t g = c->blockrows ? c->blockrows[idx] : idx; /* h * nbq + r */
+    int64_t h = g / c->nbq, r = g % c->nbq;
+    int64_t a0 = r * c->B, a1 = a0 + c->B;
+    if (a1 > c->nq) a1 = c->nq;
+    double *Er = c->E + idx * c->nb;
+    for (int64_t cc = 0; cc < c->nb; ++cc) Er[cc] = 0.0;
+    for (int64_t a = a0; a < a1; ++a) {
+        int64_t i = packed_to_token(a, c->W, c->H, c->k_anchor, c->anchors);
+        const uint16_t *qi = c->q + (h * c->n + i) * c->d;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < c->n; ++j) {
+            const uint16_t *kj = c->k + (h * c->n + j) * c->d;
+            double dot = 0.0;
+            for (int u = 0; u < c->d; ++u) dot += bf16_to_double(qi[u]) * bf16_to_double(kj[u]);
+            s[j] = c->scale * dot;
+            if (s[j] > m) m = s[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < c->n; ++j) l += exp(s[j] - m);
+        double lse_i = m + log(l);
+        for (int64_t j = 0; j < c->n; ++j) Er[j / c->B] += exp(s[j] - lse_i);
+    }
+    for (int64_t cc = 0; cc < c->nb; ++cc) Er[cc] /= (double)(a1 - a0);
+}
+
+/* E: [n_blockrows][nb] for blockrows h*nbq + r (all of them when NULL). */
+int oracle_anchor_block_energy(const uint16_t *q, const uint16_t *k, int heads, int F, int H, int W, int d,
+                               int B, int k_anchor, double scale, const int64_t *blockrows,
+                               int64_t n_blockrows, double *E, int threads) {
+    if (k_anchor < 1 || k_anchor > H) return -1;
+    int *anchors = (int *)malloc(sizeof(int) * (size_t)k_anchor);
+    oracle_anchor_rows(H, k_anchor, anchors);
+    int64_t n = (int64_t)F * H * W, nq = (int64_t)F * k_anchor * W;
+    anchor_energy_ctx c = {q, k, d, B, H, W, k_anchor, n, nq, (nq + B - 1) / B, (n + B - 1) / B, scale,
+                           anchors, blockrows, E};
+    if (!blockrows) n_blockrows = (int64_t)heads * c.nbq;
+    run_rows(anchor_energy_blockrow, &c, n_blockrows, threads, (size_t)n);
+    free(anchors);
+    return 0;
+}
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int d, B, H, W, k_anchor;
+    int64_t n, nbq, nb;
+    double scale;
+    const int *anchors, *owner;
+    const uint8_t *mask_b; /* [heads][nbq][nb] */
+    const int64_t *rows;
+    double *o, *lse;
+} rep_masked_ctx;
+
+static void rep_masked_row(void *vctx, int64_t idx, double *s) {
+    rep_masked_ctx *c = (rep_masked_ctx *)vctx;
+    int64_t gi = c->rows ? c->rows[idx] : idx;
+    int64_t h = gi / c->n, t = gi % c->n;
+    int64_t hw = (int64_t)c->H * c->W;
+    int64_t f = t / hw, rem = t % hw;
+    int64_t row = rem / c->W, col = rem % c->W;
+    int64_t jn = c->owner[row];                         /* nearest anchor */
+    int64_t a = f * (int64_t)c->k_anchor * c->W + jn * c->W + col; /* its packed index */
+    int64_t src = f * hw + (int64_t)c->anchors[jn] * c->W + col;   /* its token */
+    const uint8_t *mrow = c->mask_b + (h * c->nbq + a / c->B) * c->nb;
+    const uint16_t *qi = c->q + (h * c->n + src) * c->d;
+    double *oi = c->o + idx * c->d;
+    double m = -INFINITY;
+    int64_t cnt = 0;
+    for (int64_t j = 0; j < c->n; ++j) {
+        if (!mrow[j / c->B]) continue;
+        const uint16_t *kj = c->k + (h * c->n + j) * c->d;
+        double dot = 0.0;
+        for (int u = 0; u < c->d; ++u) dot += bf16_to_double(qi[u]) * bf16_to_double(kj[u]);
+        s[cnt] = c->scale * dot;
+        if (s[cnt] > m) m = s[cnt];
+        ++cnt;
+    }
+    for (int u = 0; u < c->d; ++u) oi[u] = 0.0;
+    if (cnt == 0) {
+        c->lse[idx] = -INFINITY;
+        return;
+    }
+    double l = 0.0;
+    cnt = 0;
+    for (int64_t j = 0; j < c->n; ++j) {
+        if (!mrow[j / c->B]) continue;
+        double p = exp(s[cnt++] - m);
+        l += p;
+        const uint16_t *vj = c->v + (h * c->n + j) * c->d;
+        for (int u = 0; u < c->d; ++u) oi[u] += p * bf16_to_double(vj[u]);
+    }
+    for (int u = 0; u < c->d; ++u) oi[u] /= l;
+    c->lse[idx] = m + log(l);
+}
+
+int oracle_repeat_attention_masked(const uint16_t *q, const uint16_t *k, const uint16_t *v, int heads, int F,
+                                   int H, int W, int d, int B, int k_anchor, double scale,
+                                   const uint8_t *mask_b, const int64_t *rows, int64_t n_rows, double *o,
+                                   double *lse, int threads) {
+    if (k_anchor < 1 || k_anchor > H) return -1;
+    int *anchors = (int *)malloc(sizeof(int) * (size_t)k_anchor);
+    int *owner = (int *)malloc(sizeof(int) * (size_t)H);
+    oracle_anchor_rows(H, k_anchor, anchors);
+    oracle_nearest_anchor(H, k_anchor, anchors, owner);
+    int64_t n = (int64_t)F * H * W, nq = (int64_t)F * k_anchor * W;
+    rep_masked_ctx c = {q, k, v, d, B, H, W, k_anchor, n, (nq + B - 1) / B, (n + B - 1) / B, scale,
+                        anchors, owner, mask_b, rows, o, lse};
+    if (!rows) n_rows = (int64_t)heads * n;
+    run_rows(rep_masked_row, &c, n_rows, threads, (size_t)n);
+    free(anchors);
+    free(owner);
+    return 0;
+}
