@@ -267,7 +267,406 @@ def graph_time(fn, reps, stream):
     return ms
 
 
-TRAFFIC_PER_TILE = 565.24e6 / 514058  # dram bytes per kept tile, measured (see the roofline block)
+# DRAM bytes per kept tile of the attention kernel: one ncu capture of the
+# 5-head Wan-720p launch (heads 0-3 block-sparse, head 4 repeated), 565.2 MB
+# of dram__bytes_read.sum + dram__bytes_write.sum over its 514 058 kept tiles;
+# the roofline's traffic scales it by the tiles of the timed launch.
+TRAFFIC_PER_TILE = 565.24e6 / 514058
+
+
+def frac_of(achieved, pk, key):
+    return achieved / pk[key] if pk.get(key) else None
+
+
+def calibrate(binding, wl, n_in, eps, dev, stream, first_input=0):
+    """Calibration of one (t, l) on the device: every input through the
+    single-pass energy kernel with fused eps selection, masks folded into
+    counts; the tie-affected selections (1e-6) are counted. Returns (counts,
+    info)."""
+    heads, nb, n = wl.heads, wl.nb, wl.n
+    counts = torch.zeros((heads, nb, nb), dtype=torch.uint16, device=dev)
+    tie = torch.empty((heads, nb), dtype=torch.uint8, device=dev)
+    ws = torch.empty(binding.energy_workspace_size(heads, n), dtype=torch.uint8, device=dev)
+    ms, ties = 0.0, 0
+    for p in range(first_input, first_input + n_in):
+        q, k, _ = synth.qkv(wl, p, with_v=False, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        binding.block_energy_1pass(q, k, eps=eps, energy=False, counts=counts, ws=ws, tie=tie, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        ms += e0.elapsed_time(e1)
+        ties += int(tie.sum().item())
+    binding.check_status(what=f"calibration of {wl.name}")
+    f_alg = 2.0 * D * n * n * heads  # one S = Q K^T per input
+    info = {"inputs": n_in, "eps": eps, "rho": 0.5,
+            "energy_ms_per_input": ms / n_in, "energy_tflops": f_alg / (ms / n_in * 1e-3) / 1e12,
+            "tie_affected_selections": ties, "selections": n_in * heads * nb, "tie_window": binding.TIE_WINDOW,
+            "kernel": "calibatt_block_energy_1pass (fused eps selection, counts and tie flags)"}
+    return counts, info
+
+
+def skip_lists(binding, wl, dev, stream):
+    """Masks and skip lists of a workload: random block masks (Wan-720p) or
+    calibration on the GPU over the workload's seeded inputs."""
+    if wl.name == "wan720":
+        masks = synth.random_block_masks(synth.WORKLOADS["wan720"])[:wl.heads]
+        counts = torch.from_numpy(masks.astype(np.int16)).to(dev).view(torch.uint16)
+        _, row_ptr, col_idx, _ = binding.aggregate_masks(counts, 1, 0.5)
+        calib = {"source": "random per-head block masks (Beta(2,3) keep rates, diagonal and first frame kept)"}
+    else:
+        n_cal, eps_cal = synth.CALIBRATION[wl.name]
+        counts, calib = calibrate(binding, wl, n_cal, eps_cal, dev, stream)
+        mask_d, row_ptr, col_idx, _ = binding.aggregate_masks(counts, n_cal, 0.5)
+        masks = mask_d.cpu().numpy()
+        calib["source"] = "calibrated on the GPU"
+    binding.check_status(what="skip lists")
+    return masks, row_ptr, col_idx, calib
+
+
+def dense_run(binding, q, k, v, o, lse, heads, nb, dev, stream, reps):
+    """The same kernel with every block kept on every head (0 % sparsity)."""
+    full = torch.ones((heads, nb, nb), dtype=torch.int16, device=dev).view(torch.uint16)
+    _, rp_full, ci_full, _ = binding.aggregate_masks(full, 1, 0.5)
+    rp_full_h = rp_full.cpu().numpy()
+    work_full = torch.from_numpy(binding.balance_plan(binding.build_plan(rp_full_h, heads, nb), rp_full_h, heads,
+                                                      nb)).to(dev)
+
+    def dense_call():
+        binding.sparse_attn_fwd(q, k, v, rp_full, ci_full, work_full, o=o, lse=lse, stream=stream)
+
+    dense_call()
+    ms = cuda_time(dense_call, reps, stream)
+    binding.check_status(what="dense")
+    return ms
+
+
+def library_dense(q, k, v, stream, reps, f_dense):
+    """Context, not this library's path: the same dense attention by the cuDNN
+    backend of torch's scaled_dot_product_attention, timed the same way."""
+    try:
+        import torch.nn.functional as F
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+
+        def library_call():
+            with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+                return F.scaled_dot_product_attention(q[None], k[None], v[None])
+
+        with torch.cuda.stream(stream):
+            library_call()
+            lib_ms = cuda_time(library_call, reps, stream)
+        return {"kernel": "torch scaled_dot_product_attention, cuDNN backend, all blocks kept",
+                "ms": lib_ms, "tflops": f_dense / (lib_ms * 1e-3) / 1e12}
+    except Exception as exc:  # the backend may be missing: report why
+        return {"unavailable": str(exc)[:200]}
+
+
+class Step:
+    """One attention call of a workload through calibatt_mixed_attn_fwd:
+    block-sparse heads over their skip lists and repeated heads' anchor rows
+    in one persistent launch (after the anchor gather)."""
+
+    def __init__(self, binding, wl, masks, row_ptr, col_idx, dev, stream, input_idx=1000, rep_heads=None):
+        self.b, self.wl, self.stream = binding, wl, stream
+        heads, nb, n = wl.heads, wl.nb, wl.n
+        self.rep = list(wl.repeat_heads) if rep_heads is None else list(rep_heads)
+        self.sparse_heads = [h for h in range(heads) if h not in self.rep]
+        self.masks, self.row_ptr, self.col_idx = masks, row_ptr, col_idx
+        self.row_ptr_h = row_ptr.cpu().numpy()
+        self.q, self.k, self.v = synth.qkv(wl, input_idx, device=dev)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((heads, n), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(binding.repeat_workspace_size(max(len(self.rep), 1), wl.F, wl.H, wl.W,
+                                                                wl.k_anchor), 256), dtype=torch.uint8, device=dev)
+        self.rep_t = torch.tensor(self.rep, dtype=torch.int32, device=dev)
+        work = binding.build_mixed_plan(self.row_ptr_h, heads, nb, self.rep, wl.F, wl.H, wl.W, wl.k_anchor)
+        self.work = torch.from_numpy(binding.balance_plan(work, self.row_ptr_h, heads, nb)).to(dev)
+        self.f_sparse = sparse_flops(masks, self.sparse_heads, n)
+        self.f_rep = repeat_flops(wl, len(self.rep))
+        self.flops = self.f_sparse + self.f_rep
+        self.kept_frac = float(np.mean([masks[h].mean() for h in self.sparse_heads])) if self.sparse_heads else 1.0
+        self.tiles = int(sum(int(masks[h].sum()) for h in self.sparse_heads)) + \
+            len(self.rep) * -(-wl.F * wl.k_anchor * wl.W // 128) * nb
+        self.launches = 1 + (1 if self.rep else 0)
+
+    def __call__(self):
+        wl = self.wl
+        self.b.mixed_attn_fwd(self.q, self.k, self.v, wl.F, wl.H, wl.W, self.row_ptr, self.col_idx, self.rep_t,
+                              self.work, wl.k_anchor, o=self.o, lse=self.lse, ws=self.ws, stream=self.stream)
+
+    def summary(self, ms, dense_ms, pk, library=None):
+        wl = self.wl
+        tflops = self.flops / (ms * 1e-3) / 1e12
+        out = {"shape": f"{wl.heads} heads x N={wl.n} (F={wl.F},H={wl.H},W={wl.W}), d={D}, "
+                        f"{len(self.sparse_heads)} block-sparse + {len(self.rep)} repeated (k={wl.k_anchor})",
+               "ms_per_call": ms, "kept_tile_tflops": tflops,
+               "frac_of_bf16_burst": frac_of(tflops, pk, "bf16_tflops"),
+               "frac_of_bf16_sustained": frac_of(tflops, pk, "bf16_tflops_sustained"),
+               "kept_tile_flops": self.flops, "kept_tiles": self.tiles,
+               "block_sparsity": 1.0 - self.kept_frac, "kept_block_fraction": self.kept_frac}
+        if dense_ms is not None:
+            f_dense = float(4 * D * wl.n * wl.n * wl.heads)
+            out.update({"dense_ms": dense_ms, "dense_tflops": f_dense / (dense_ms * 1e-3) / 1e12,
+                        "speedup_vs_dense": dense_ms / ms})
+        if library is not None:
+            out["library_dense"] = library
+        return out
+
+
+def attention_config(binding, name, dev, pk, reps, with_library):
+    """Skip lists (calibrated or random), then one attention call timed, and
+    the same kernel at 0 % sparsity, on a stream of its own (CUDA graphs time
+    the launch-bound small workloads; they cannot capture the legacy stream)."""
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        out, step = _attention_config(binding, name, dev, stream, pk, reps, with_library)
+    torch.cuda.synchronize()
+    return out, step
+
+
+def _attention_config(binding, name, dev, stream, pk, reps, with_library):
+    wl = synth.WORKLOADS[name]
+    masks, row_ptr, col_idx, calib = skip_lists(binding, wl, dev, stream)
+    step = Step(binding, wl, masks, row_ptr, col_idx, dev, stream)
+    for _ in range(3):
+        step()
+    timer = graph_time if wl.n * wl.heads < 1_000_000 else cuda_time
+    ms = timer(step, reps, stream)
+    binding.check_status(what=name)
+    dense_ms = dense_run(binding, step.q, step.k, step.v, step.o, step.lse, wl.heads, wl.nb, dev, stream,
+                         max(2, reps // 3)) if wl.n * wl.heads >= 1_000_000 else None
+    if dense_ms is None:
+        # launch-bound sizes: the dense run through a graph as well
+        full = torch.ones((wl.heads, wl.nb, wl.nb), dtype=torch.int16, device=dev).view(torch.uint16)
+        _, rpf, cif, _ = binding.aggregate_masks(full, 1, 0.5)
+        rpf_h = rpf.cpu().numpy()
+        wf = torch.from_numpy(binding.build_plan(rpf_h, wl.heads, wl.nb)).to(dev)
+        dense_ms = graph_time(lambda: binding.sparse_attn_fwd(step.q, step.k, step.v, rpf, cif, wf, o=step.o,
+                                                              lse=step.lse, stream=stream), reps, stream)
+    lib = library_dense(step.q, step.k, step.v, stream, max(2, reps // 3),
+                        float(4 * D * wl.n * wl.n * wl.heads)) if with_library else None
+    step()  # the dense run wrote the same output buffers: restore the call's result
+    out = step.summary(ms, dense_ms, pk, lib)
+    out["skip_lists"] = calib
+    return out, step
+
+
+def calibration_kernels(binding, wl, q, k, dev, stream, pk):
+    """The calibration kernels on one input of the full Wan-720p shape (all
+    heads): both energy kernels with fused selection, standalone selection,
+    aggregation into the skip list, pixel-row profiles and the spatial score.
+    The bandwidth-bound ones are timed through CUDA graphs and reported
+    against the measured HBM copy bandwidth."""
+    heads, nb, n = wl.heads, wl.nb, wl.n
+    hbm = pk.get("hbm_gbs")
+    lse_ws = torch.empty((heads, nb * 128), dtype=torch.float32, device=dev)
+    energy = torch.empty((heads, nb, nb), dtype=torch.float32, device=dev)
+    cmask = torch.empty((heads, nb, nb), dtype=torch.uint8, device=dev)
+    ccounts = torch.zeros((heads, nb, nb), dtype=torch.uint16, device=dev)
+
+    def energy_call():
+        binding.block_energy(q, k, eps=0.9, energy=energy, mask=cmask, counts=ccounts, lse_ws=lse_ws, stream=stream)
+
+    energy_call()
+    e_ms = cuda_time(energy_call, 2, stream)
+    ews = torch.empty(binding.energy_workspace_size(heads, n), dtype=torch.uint8, device=dev)
+
+    def energy1_call():
+        binding.block_energy_1pass(q, k, eps=0.9, energy=energy, mask=cmask, counts=ccounts, ws=ews, stream=stream)
+
+    energy1_call()
+    e1_ms = cuda_time(energy1_call, 2, stream)
+    del ews
+    f_alg = float(2 * D * n * n * heads)  # one S = Q K^T per input
+    gstream = torch.cuda.Stream()
+    tie = torch.empty((heads, nb), dtype=torch.uint8, device=dev)
+
+    def select_call():
+        binding.select_mask(energy, 0.9, mask=cmask, kept=False, tie=tie, stream=torch.cuda.current_stream())
+
+    with torch.cuda.stream(gstream):
+        s_ms = graph_time(select_call, 20, gstream)
+    sel_bytes = heads * nb * nb * (4 + 1) + heads * nb
+    agg_ws = torch.empty(binding.load().calibatt_aggregate_workspace_size(heads, nb), dtype=torch.uint8, device=dev)
+    am = torch.empty((heads, nb, nb), dtype=torch.uint8, device=dev)
+    arp = torch.empty(heads * nb + 1, dtype=torch.int32, device=dev)
+    aci = torch.empty(heads * nb * nb, dtype=torch.int32, device=dev)
+    annz = torch.zeros(1, dtype=torch.int64, device=dev)
+    lib = binding.load()
+
+    def agg_call():
+        lib.calibatt_aggregate_masks(binding._ptr(ccounts), 64, heads, nb, 0.5, binding._ptr(am),
+                                     binding._ptr(arp), binding._ptr(aci), aci.numel(), binding._ptr(annz),
+                                     binding._ptr(agg_ws), agg_ws.numel(),
+                                     binding._stream(torch.cuda.current_stream()))
+
+    with torch.cuda.stream(gstream):
+        a_ms = graph_time(agg_call, 20, gstream)
+    pix = torch.empty((heads, wl.F * wl.H, nb), dtype=torch.float32, device=dev)
+
+    def pix_call():
+        binding.pixel_row_energy(q, k, wl.F, wl.H, wl.W, pix=pix, lse_ws=lse_ws, stream=stream)
+
+    pix_call()
+    p_ms = cuda_time(pix_call, 2, stream)
+    sscore = torch.empty(heads, dtype=torch.float32, device=dev)
+    sflag = torch.empty(heads, dtype=torch.uint8, device=dev)
+
+    def score_call():
+        binding.spatial_score(pix, wl.F, wl.H, wl.k_anchor, score=sscore, flag=sflag,
+                              stream=torch.cuda.current_stream())
+
+    with torch.cuda.stream(gstream):
+        sc_ms = graph_time(score_call, 20, gstream)
+    binding.check_status(what="calibration kernels")
+    kept_agg = int(annz.item())
+    agg_bytes = heads * nb * nb * (2 + 1) + kept_agg * 4 + (heads * nb + 1) * 4
+    score_bytes = heads * wl.F * wl.H * nb * 4  # every profile row read once
+    out = {
+        "shape": f"{heads} heads x N={n}",
+        "energy_2pass_ms": e_ms, "energy_2pass_tflops_algorithmic": f_alg / (e_ms * 1e-3) / 1e12,
+        "energy_2pass_tflops_issued": 2 * f_alg / (e_ms * 1e-3) / 1e12,
+        "energy_1pass_ms": e1_ms, "energy_1pass_tflops": f_alg / (e1_ms * 1e-3) / 1e12,
+        "select_ms": s_ms, "select_gbs": sel_bytes / (s_ms * 1e-3) / 1e9,
+        "select_bytes": sel_bytes,
+        "aggregate_ms": a_ms, "aggregate_gbs": agg_bytes / (a_ms * 1e-3) / 1e9, "aggregate_bytes": agg_bytes,
+        "eps": 0.9, "kept_fraction_at_eps": float(cmask.float().mean().item()),
+        "tie_affected_rows_at_eps": int(tie.sum().item()),
+        "pixel_row_energy_ms": p_ms, "pixel_row_energy_tflops_issued": 2 * f_alg / (p_ms * 1e-3) / 1e12,
+        "spatial_score_ms": sc_ms, "spatial_score_gbs": score_bytes / (sc_ms * 1e-3) / 1e9,
+        "spatial_flagged_heads": np.nonzero(sflag.cpu().numpy())[0].tolist(),
+    }
+    if hbm:
+        for key in ("select", "aggregate", "spatial_score"):
+            out[key + "_frac_of_hbm"] = out[key + "_gbs"] / hbm
+    return out
+
+
+def calib_sweep(binding, dev, stream, pk, n_in):
+    """The calibration sweep workload: 40 heads of the Wan-720p shape, n_in
+    inputs (64), eps in {0.84, 0.9, 0.95, 0.99}, rho = 0.5. Each input's
+    energies come from the single-pass kernel (the full P never reaches HBM)
+    and stay on the device; the standalone selection then runs at every eps,
+    folding each mask into that eps's counts, and the counts are aggregated
+    into the skip list."""
+    wl = synth.WORKLOADS["calib720"]
+    heads, nb, n = wl.heads, wl.nb, wl.n
+    hbm = pk.get("hbm_gbs")
+    ws = torch.empty(binding.energy_workspace_size(heads, n), dtype=torch.uint8, device=dev)
+    energies, e_ms = [], 0.0
+    fused_ms = None
+    for p in range(n_in):
+        q, k, _ = synth.qkv(wl, p, with_v=False, device=dev)
+        E = torch.empty((heads, nb, nb), dtype=torch.float32, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        binding.block_energy_1pass(q, k, energy=E, ws=ws, stream=stream)
+        e1.record(stream)
+        if p == 0:
+            # the same pass with the selection fused (eps = 0.9), for its cost
+            fm = torch.empty((heads, nb, nb), dtype=torch.uint8, device=dev)
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            binding.block_energy_1pass(q, k, eps=0.9, energy=False, mask=fm, ws=ws, stream=stream)
+            f1.record(stream)
+            f1.synchronize()
+            fused_ms = f0.elapsed_time(f1)
+            del fm
+        e1.synchronize()
+        e_ms += e0.elapsed_time(e1)
+        energies.append(E)
+        del q, k
+    del ws
+    f_alg = float(2 * D * n * n * heads)
+    out = {"shape": f"{heads} heads x N={n} (F={wl.F},H={wl.H},W={wl.W}), d={D}", "inputs": n_in, "rho": 0.5,
+           "energy_kernel": "calibatt_block_energy_1pass",
+           "energy_ms_per_input": e_ms / n_in, "energy_tflops": f_alg / (e_ms / n_in * 1e-3) / 1e12,
+           "energy_fused_select_ms": fused_ms,
+           "energy_fused_select_tflops": f_alg / (fused_ms * 1e-3) / 1e12 if fused_ms else None, "eps": {}}
+    agg_ws = torch.empty(binding.load().calibatt_aggregate_workspace_size(heads, nb), dtype=torch.uint8, device=dev)
+    tie = torch.empty((heads, nb), dtype=torch.uint8, device=dev)
+    cells = heads * nb * nb
+    for eps in (0.84, 0.9, 0.95, 0.99):
+        counts = torch.zeros((heads, nb, nb), dtype=torch.uint16, device=dev)
+        ties = 0
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tie_sum = torch.zeros((), dtype=torch.int64, device=dev)
+        torch.cuda.synchronize()
+        s0.record(stream)
+        for E in energies:
+            binding.select_mask(E, eps, mask=False, kept=False, counts=counts, tie=tie, stream=stream)
+            with torch.cuda.stream(stream):
+                tie_sum += tie.sum()
+        s1.record(stream)
+        s1.synchronize()
+        sel_ms = s0.elapsed_time(s1) / n_in
+        ties = int(tie_sum.item())
+        kept_cells = int((counts.view(torch.int16).to(torch.int32) & 0xFFFF).sum().item())
+        mask, row_ptr, col_idx, nnz = binding.aggregate_masks(counts, n_in, 0.5, ws=agg_ws, stream=stream)
+        nnz_v = int(nnz.item())
+
+        def agg_call():
+            binding.aggregate_masks(counts, n_in, 0.5, ws=agg_ws, stream=torch.cuda.current_stream(), trim=False)
+
+        gstream = torch.cuda.Stream()
+        with torch.cuda.stream(gstream):
+            a_ms = graph_time(agg_call, 10, gstream)
+        binding.check_status(what=f"sweep eps {eps}")
+        # selection: the energies read, plus each kept block's count read and written
+        sel_bytes = cells * 4 + (kept_cells / n_in) * 4 + heads * nb
+        agg_bytes = cells * (2 + 1) + nnz_v * 4 + (heads * nb + 1) * 4
+        e = {"block_sparsity": 1.0 - nnz_v / cells, "kept_blocks": nnz_v,
+             "mean_kept_fraction_per_input": kept_cells / n_in / cells,
+             "tie_affected_selections": ties, "selections": n_in * heads * nb, "tie_window": binding.TIE_WINDOW,
+             "select_ms_per_input": sel_ms, "select_gbs": sel_bytes / (sel_ms * 1e-3) / 1e9,
+             "aggregate_ms": a_ms, "aggregate_gbs": agg_bytes / (a_ms * 1e-3) / 1e9}
+        if hbm:
+            e["select_frac_of_hbm"] = e["select_gbs"] / hbm
+            e["aggregate_frac_of_hbm"] = e["aggregate_gbs"] / hbm
+        out["eps"][str(eps)] = e
+        del counts, mask, row_ptr, col_idx
+    del energies
+    return out
+
+
+def fp8_probe(binding, name, n_in, dev, stream):
+    """Calibration with q and k rounded to FP8 e4m3 (the operands an FP8
+    Q K^T would see; products are exact in fp32 either way) against the same
+    calibration in bf16: energy error, selections that change, aggregated
+    cells that change."""
+    wl = synth.WORKLOADS[name]
+    heads, nb, n = wl.heads, wl.nb, wl.n
+    eps = synth.CALIBRATION[name][1]
+    ws = torch.empty(binding.energy_workspace_size(heads, n), dtype=torch.uint8, device=dev)
+    c16 = torch.zeros((heads, nb, nb), dtype=torch.uint16, device=dev)
+    c8 = torch.zeros_like(c16)
+    t16 = torch.empty((heads, nb), dtype=torch.uint8, device=dev)
+    max_rel, max_abs_rowmax, rows_diff, rows_diff_untied, rows = 0.0, 0.0, 0, 0, 0
+    for p in range(n_in):
+        q, k, _ = synth.qkv(wl, p, with_v=False, device=dev)
+        E16, m16, _, _, _, _ = binding.block_energy_1pass(q, k, eps=eps, mask=torch.empty(
+            (heads, nb, nb), dtype=torch.uint8, device=dev), counts=c16, ws=ws, tie=t16, stream=stream)
+        q8 = q.to(torch.float8_e4m3fn).to(torch.bfloat16)
+        k8 = k.to(torch.float8_e4m3fn).to(torch.bfloat16)
+        E8, m8, _, _, _ = binding.block_energy_1pass(q8, k8, eps=eps, mask=torch.empty(
+            (heads, nb, nb), dtype=torch.uint8, device=dev), counts=c8, ws=ws, stream=stream)
+        rowmax = E16.amax(-1, keepdim=True)
+        sig = E16 >= 1e-3 * rowmax
+        max_rel = max(max_rel, float(((E8 - E16).abs() / E16.clamp_min(1e-30))[sig].max().item()))
+        max_abs_rowmax = max(max_abs_rowmax, float(((E8 - E16).abs() / rowmax).max().item()))
+        d = (m16 != m8).any(-1)
+        rows_diff += int(d.sum().item())
+        rows_diff_untied += int((d & (t16 == 0)).sum().item())
+        rows += heads * nb
+    a16, _, _, _ = binding.aggregate_masks(c16, n_in, 0.5, stream=stream)
+    a8, _, _, _ = binding.aggregate_masks(c8, n_in, 0.5, stream=stream)
+    binding.check_status(what="fp8 probe")
+    return {"inputs": n_in, "eps": eps, "rounding": "q and k to float8_e4m3fn (no scaling), energies otherwise bf16",
+            "max_rel_energy_error_on_entries_above_1e-3_rowmax": max_rel,
+            "max_abs_energy_error_over_rowmax": max_abs_rowmax,
+            "selection_rows_changed": rows_diff, "selection_rows_changed_not_tie_affected_at_1e-6": rows_diff_untied,
+            "selection_rows": rows, "aggregated_cells_changed": int((a16 != a8).sum().item()),
+            "aggregated_cells": heads * nb * nb}
 
 
 def run_ours(args, world, rank, local):
@@ -280,76 +679,35 @@ def run_ours(args, world, rank, local):
         wl = dataclasses.replace(wl, heads=args.heads, repeat_heads=tuple(h for h in wl.repeat_heads if h < args.heads))
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
+    pk, pk_src = peaks()
     n, nb, heads = wl.n, wl.nb, wl.heads
     rep_heads = list(wl.repeat_heads)
     sparse_heads = [h for h in range(heads) if h not in rep_heads]
 
-    # inputs: resident in HBM before the timed region
-    if args.workload == "wan720":
-        # random per-head masks at 62.5 % sparsity; skip lists built on the GPU
-        # by the aggregation kernel (one input, rho 0.5)
-        masks = synth.random_block_masks(synth.WORKLOADS["wan720"])[:heads]
-        counts = torch.from_numpy(masks.astype(np.int16)).to(dev).view(torch.uint16)
-        mask_d, row_ptr, col_idx, _ = binding.aggregate_masks(counts, 1, 0.5)
-    else:
-        # masks calibrated on the GPU over the workload's seeded inputs
-        n_cal, eps_cal = synth.CALIBRATION[args.workload]
-        counts = torch.zeros((heads, nb, nb), dtype=torch.uint16, device=dev)
-        cws = torch.empty(binding.energy_workspace_size(heads, n), dtype=torch.uint8, device=dev)
-        for pi in range(n_cal):
-            qc, kc, _ = synth.qkv(wl, pi, with_v=False, device=dev)
-            binding.block_energy_1pass(qc, kc, eps=eps_cal, energy=False, counts=counts, ws=cws)
-            del qc, kc
-        del cws
-        mask_d, row_ptr, col_idx, _ = binding.aggregate_masks(counts, n_cal, 0.5)
-        masks = mask_d.cpu().numpy()
-    binding.check_status(what="skip lists")
-    q, k, v = synth.qkv(wl, 1000 + rank, device=dev)
+    # inputs and skip lists: resident in HBM before the timed region
+    masks, row_ptr, col_idx, calib_info = skip_lists(binding, wl, dev, stream)
     row_ptr_h = row_ptr.cpu().numpy()
-    head_active = np.array([h not in rep_heads for h in range(heads)], np.uint8)
-    # every work list is laid out for the device's worker slots (balanced
-    # static schedule; any order gives the same output)
-    work = torch.from_numpy(binding.balance_plan(binding.build_plan(row_ptr_h, heads, nb, head_active), row_ptr_h,
-                                                 heads, nb)).to(dev)
-    rep_t = torch.tensor(rep_heads, dtype=torch.int32, device=dev)
-    o = torch.empty_like(q)
-    lse = torch.empty((heads, n), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(binding.repeat_workspace_size(max(len(rep_heads), 1), wl.F, wl.H, wl.W, wl.k_anchor), 256),
-                     dtype=torch.uint8, device=dev)
-
-    f_sparse = sparse_flops(masks, sparse_heads, n)
-    f_rep = repeat_flops(wl, len(rep_heads))
-    f_step = f_sparse + f_rep
-    kept_frac = float(np.mean([masks[h].mean() for h in sparse_heads]))
-
-    def sparse_call():
-        binding.sparse_attn_fwd(q, k, v, row_ptr, col_idx, work, o=o, lse=lse, stream=stream)
-
-    def repeat_call():
-        if rep_heads:
-            binding.repeat_attn_fwd(q, k, v, wl.F, wl.H, wl.W, rep_t, wl.k_anchor, o=o, lse=lse, ws=ws,
-                                    stream=stream)
-
-    # the step: block-sparse and repeated heads in one persistent launch
-    # (after the anchor gather). --shard heads: one call split over the ranks
-    # by heads (balanced by kept tiles, no exchange), strong scaling
+    # --shard heads: one call split over the ranks by heads (balanced by kept
+    # tiles, no exchange), strong scaling; else a replica of the call per rank
     shard = args.shard == "heads" and world > 1
+    owner = None
     if shard:
         owner, _ = binding.shard_heads(row_ptr_h, heads, nb, rep_heads, wl.F, wl.W, wl.k_anchor, world)
-        work_np, my_rep = binding.build_rank_plan(row_ptr_h, heads, nb, rep_heads, owner, rank, wl.F, wl.H, wl.W,
-                                                  wl.k_anchor)
-        f_rank = sparse_flops(masks, [h for h in sparse_heads if owner[h] == rank], n) + repeat_flops(wl, len(my_rep))
+        my_rep = [h for h in rep_heads if owner[h] == rank]
     else:
-        work_np = binding.build_mixed_plan(row_ptr_h, heads, nb, rep_heads, wl.F, wl.H, wl.W, wl.k_anchor)
-        my_rep, f_rank = rep_heads, f_step
-    work_mixed = torch.from_numpy(binding.balance_plan(work_np, row_ptr_h, heads, nb)).to(dev)
-    my_rep_t = torch.tensor(my_rep, dtype=torch.int32, device=dev)
+        my_rep = rep_heads
+    step = Step(binding, wl, masks, row_ptr, col_idx, dev, stream, input_idx=1000 + rank, rep_heads=my_rep)
+    if shard:
+        work_np, _ = binding.build_rank_plan(row_ptr_h, heads, nb, rep_heads, owner, rank, wl.F, wl.H, wl.W,
+                                             wl.k_anchor)
+        step.work = torch.from_numpy(binding.balance_plan(work_np, row_ptr_h, heads, nb)).to(dev)
+        mine = [h for h in sparse_heads if owner[h] == rank]
+        step.flops = sparse_flops(masks, mine, n) + repeat_flops(wl, len(my_rep))
+        step.tiles = int(sum(int(masks[h].sum()) for h in mine)) + \
+            len(my_rep) * -(-wl.F * wl.k_anchor * wl.W // 128) * nb
+    f_step = sparse_flops(masks, sparse_heads, n) + repeat_flops(wl, len(rep_heads))  # the whole call
+    q, k, v, o, lse = step.q, step.k, step.v, step.o, step.lse
 
-    def step():
-        binding.mixed_attn_fwd(q, k, v, wl.F, wl.H, wl.W, row_ptr, col_idx, my_rep_t, work_mixed, wl.k_anchor, o=o,
-                               lse=lse, ws=ws, stream=stream)
-
-    launches_per_step = 1 + (1 if my_rep else 0)
     for _ in range(args.warmup):
         step()
     binding.check_status(what="warmup")
@@ -374,52 +732,38 @@ def run_ours(args, world, rank, local):
     binding.check_status(what="timed steps")
     attn_ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
     ms_step = elapsed_ms / args.steps
-
-    # the same work as two separate calls (block-sparse, then repeated heads)
-    sparse_ms = repeat_ms = None
-    if not shard:
-        sparse_ms = cuda_time(sparse_call, max(2, min(5, args.steps)), stream)
-        repeat_ms = cuda_time(repeat_call, max(2, min(5, args.steps)), stream) if rep_heads else 0.0
-        binding.check_status(what="separate calls")
     # weak scaling: every rank runs the whole call (replicas); strong: the
     # ranks share one call
     value = (1 if shard else world) * f_step / (ms_step * 1e-3) / 1e12
+    reps = max(2, min(5, args.steps))
 
-    # ---- 0 %-sparse run: the same kernel with every block kept, all 40 heads
-    full = torch.ones((heads, nb, nb), dtype=torch.int16, device=dev).view(torch.uint16)
-    _, rp_full, ci_full, _ = binding.aggregate_masks(full, 1, 0.5)
-    rp_full_h = rp_full.cpu().numpy()
-    work_full = torch.from_numpy(binding.balance_plan(binding.build_plan(rp_full_h, heads, nb), rp_full_h, heads,
-                                                      nb)).to(dev)
+    # the same work as two separate calls (block-sparse, then repeated heads)
+    separate = None
+    if not shard:
+        head_active = np.array([h not in rep_heads for h in range(heads)], np.uint8)
+        work_s = torch.from_numpy(binding.balance_plan(binding.build_plan(row_ptr_h, heads, nb, head_active),
+                                                       row_ptr_h, heads, nb)).to(dev)
 
-    def dense_call():
-        binding.sparse_attn_fwd(q, k, v, rp_full, ci_full, work_full, o=o, lse=lse, stream=stream)
+        def sparse_call():
+            binding.sparse_attn_fwd(q, k, v, row_ptr, col_idx, work_s, o=o, lse=lse, stream=stream)
 
-    dense_call()
-    dense_ms = cuda_time(dense_call, max(2, min(5, args.steps)), stream)
-    binding.check_status(what="dense")
+        def repeat_call():
+            if rep_heads:
+                binding.repeat_attn_fwd(q, k, v, wl.F, wl.H, wl.W, step.rep_t, wl.k_anchor, o=o, lse=lse, ws=step.ws,
+                                        stream=stream)
+
+        sparse_ms = cuda_time(sparse_call, reps, stream)
+        repeat_ms = cuda_time(repeat_call, reps, stream) if rep_heads else 0.0
+        binding.check_status(what="separate calls")
+        separate = {"sparse_ms": sparse_ms, "repeat_ms": repeat_ms,
+                    "sparse_tflops": step.f_sparse / (sparse_ms * 1e-3) / 1e12}
+
+    # ---- 0 %-sparse run: the same kernel with every block kept, all heads
+    dense_ms = dense_run(binding, q, k, v, o, lse, heads, nb, dev, stream, reps)
     f_dense = float(4 * D * n * n * heads)
-    del rp_full, ci_full, work_full, full
-
-    # ---- context, not this library's path: the same dense attention by the
-    # cuDNN backend of torch's scaled_dot_product_attention, timed the same way
-    library_dense = None
-    try:
-        import torch.nn.functional as F
-        from torch.nn.attention import SDPBackend, sdpa_kernel
-
-        def library_call():
-            with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
-                return F.scaled_dot_product_attention(q[None], k[None], v[None])
-
-        with torch.cuda.stream(stream):
-            library_call()
-            lib_ms = cuda_time(library_call, max(2, min(5, args.steps)), stream)
-        library_dense = {"kernel": "torch scaled_dot_product_attention, cuDNN backend, all blocks kept",
-                         "ms": lib_ms, "tflops": f_dense / (lib_ms * 1e-3) / 1e12,
-                         "step_speedup": lib_ms / ms_step}
-    except Exception as exc:  # the backend may be missing: report why
-        library_dense = {"unavailable": str(exc)[:200]}
+    lib_dense = library_dense(q, k, v, stream, reps, f_dense)
+    if "ms" in lib_dense:
+        lib_dense["step_speedup"] = lib_dense["ms"] / ms_step
 
     # ---- end to end through the C ABI with host buffers: H2D q,k,v, call, D2H o
     e2e = None
@@ -439,7 +783,6 @@ def run_ours(args, world, rank, local):
                                         stream=stream)
 
         e2e_step()
-        reps = max(2, min(5, args.steps))
         barrier(world)
         e2e_ms = max_over_ranks(cuda_time(e2e_step, reps, stream), world)
         binding.check_status(what="e2e")
@@ -466,117 +809,50 @@ def run_ours(args, world, rank, local):
         e2e["h2d_link_frac"] = e2e["h2d_bytes_per_step"] / (e2e_ms * 1e-3) / 1e9 / link_gbs
         del qh, kh, vh, oh, ws_host
 
-    # ---- calibration kernels on the same shape (8 heads of it)
-    calib = None
-    if not args.no_calib:
-        ch = min(8, heads)
-        qc, kc = q[:ch].contiguous(), k[:ch].contiguous()
-        lse_ws = torch.empty((ch, nb * 128), dtype=torch.float32, device=dev)
-        energy = torch.empty((ch, nb, nb), dtype=torch.float32, device=dev)
-        cmask = torch.empty((ch, nb, nb), dtype=torch.uint8, device=dev)
-        ccounts = torch.zeros((ch, nb, nb), dtype=torch.uint16, device=dev)
-
-        def energy_call():
-            binding.block_energy(qc, kc, eps=0.9, energy=energy, mask=cmask, counts=ccounts, lse_ws=lse_ws,
-                                 stream=stream)
-
-        energy_call()
-        e_ms = cuda_time(energy_call, 2, stream)
-        ews = torch.empty(binding.energy_workspace_size(ch, n), dtype=torch.uint8, device=dev)
-
-        def energy1_call():
-            binding.block_energy_1pass(qc, kc, eps=0.9, energy=energy, mask=cmask, counts=ccounts, ws=ews,
-                                       stream=stream)
-
-        energy1_call()
-        e1_ms = cuda_time(energy1_call, 2, stream)
-        del ews
-        f_energy_alg = float(2 * D * n * n * ch)  # one S = Q K^T per input
-        f_energy_issued = 2 * f_energy_alg        # two passes recompute S
-
-        gstream = torch.cuda.Stream()
-
-        def select_call():
-            binding.select_mask(energy, 0.9, mask=cmask, kept=False, stream=torch.cuda.current_stream())
-
-        with torch.cuda.stream(gstream):
-            s_ms = graph_time(select_call, 20, gstream)
-        sel_bytes = ch * nb * nb * (4 + 1)
-        agg_ws = torch.empty(binding.load().calibatt_aggregate_workspace_size(ch, nb), dtype=torch.uint8, device=dev)
-        am = torch.empty((ch, nb, nb), dtype=torch.uint8, device=dev)
-        arp = torch.empty(ch * nb + 1, dtype=torch.int32, device=dev)
-        aci = torch.empty(ch * nb * nb, dtype=torch.int32, device=dev)
-        annz = torch.zeros(1, dtype=torch.int64, device=dev)
-        lib = binding.load()
-
-        def agg_call():
-            lib.calibatt_aggregate_masks(binding._ptr(ccounts), 64, ch, nb, 0.5, binding._ptr(am),
-                                         binding._ptr(arp), binding._ptr(aci), aci.numel(), binding._ptr(annz),
-                                         binding._ptr(agg_ws), agg_ws.numel(),
-                                         binding._stream(torch.cuda.current_stream()))
-
-        with torch.cuda.stream(gstream):
-            a_ms = graph_time(agg_call, 20, gstream)
-        # spatial repetition: pixel-row profiles (same two passes, plus the
-        # profile atomics) and the per-head score
-        pix = torch.empty((ch, wl.F * wl.H, nb), dtype=torch.float32, device=dev)
-
-        def pix_call():
-            binding.pixel_row_energy(qc, kc, wl.F, wl.H, wl.W, pix=pix, lse_ws=lse_ws, stream=stream)
-
-        pix_call()
-        p_ms = cuda_time(pix_call, 2, stream)
-        sscore = torch.empty(ch, dtype=torch.float32, device=dev)
-        sflag = torch.empty(ch, dtype=torch.uint8, device=dev)
-
-        def score_call():
-            binding.spatial_score(pix, wl.F, wl.H, wl.k_anchor, score=sscore, flag=sflag,
-                                  stream=torch.cuda.current_stream())
-
-        with torch.cuda.stream(gstream):
-            sc_ms = graph_time(score_call, 20, gstream)
-        binding.check_status(what="calibration")
-        kept_agg = int(annz.item())
-        agg_bytes = ch * nb * nb * (2 + 1 + 1) + kept_agg * 4 + (ch * nb + 1) * 4 * 3
-        calib = {
-            "shape": f"{ch} heads x N={n}",
-            "energy_ms": e_ms, "energy_tflops_algorithmic": f_energy_alg / (e_ms * 1e-3) / 1e12,
-            "energy_tflops_issued": f_energy_issued / (e_ms * 1e-3) / 1e12,
-            "energy_1pass_ms": e1_ms, "energy_1pass_tflops": f_energy_alg / (e1_ms * 1e-3) / 1e12,
-            "select_ms": s_ms, "select_gbs": sel_bytes / (s_ms * 1e-3) / 1e9,
-            "aggregate_ms": a_ms, "aggregate_gbs": agg_bytes / (a_ms * 1e-3) / 1e9,
-            "eps": 0.9, "kept_fraction_at_eps": float(cmask.float().mean().item()),
-            "pixel_row_energy_ms": p_ms, "pixel_row_energy_tflops_issued": f_energy_issued / (p_ms * 1e-3) / 1e12,
-            "spatial_score_ms": sc_ms,
-            "spatial_score_gbs": ch * wl.F * (wl.H - wl.k_anchor) * nb * 8 / (sc_ms * 1e-3) / 1e9,
-            "spatial_flagged_heads": np.nonzero(sflag.cpu().numpy())[0].tolist(),
-        }
-        del qc, kc, lse_ws, energy, cmask, ccounts, pix
-
     # ---- roofline of the dominant kernel: the attention kernel of the step
     # (block-sparse and repeated heads in one launch; its event window also
     # holds the short anchor-gather launch before it)
-    pk, pk_src = peaks()
     long_run = elapsed_ms > 1000.0
     peak = pk.get("bf16_tflops_sustained" if long_run else "bf16_tflops")
-    achieved = f_rank / (attn_ms * 1e-3) / 1e12
+    achieved = step.flops / (attn_ms * 1e-3) / 1e12
     kname = ("attn_kernel<attention> (%d block-sparse + %d repeated heads, one launch; window includes the "
              "anchor gather)" % (len(sparse_heads), len(rep_heads)))
     if shard:
         kname += "; rank 0 share of the heads"
-    # DRAM traffic per launch: the given figure, else the bytes per kept tile
-    # of the one ncu capture (profiles/attn_kernel_wan720_5heads_ncu_full.md:
-    # 565.2 MB over 514 058 kept tiles) times the tiles of this launch
-    mine = [h for h in sparse_heads if not shard or owner[h] == rank]
-    tiles = int(sum(int(masks[h].sum()) for h in mine)) + len(my_rep) * -(-wl.F * wl.k_anchor * wl.W // 128) * nb
-    traffic = args.traffic_bytes if args.traffic_bytes else TRAFFIC_PER_TILE * tiles
+    traffic = args.traffic_bytes if args.traffic_bytes else TRAFFIC_PER_TILE * step.tiles
     roofline = {"bound": "tensor", "kernel": kname,
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{pk_src} {'sustained' if long_run else 'burst'} bf16",
                 "traffic": traffic,
                 "traffic_source": "given" if args.traffic_bytes else
-                "ncu dram bytes of a 5-head capture, scaled by kept tiles (%d in this launch)" % tiles,
+                "ncu dram bytes per kept tile of a 5-head capture, scaled by the %d kept tiles of this launch"
+                % step.tiles,
                 "algorithmic_bytes": 4.0 * heads * n * D * 2}
+
+    # ---- the other workloads, the calibration kernels and the sweep (rank 0
+    # of a one-GPU run; each is timed on its own after the timed region)
+    configs = {args.workload: step.summary(ms_step, dense_ms, pk, lib_dense)}
+    configs[args.workload]["skip_lists"] = calib_info
+    calib = sweep = fp8 = tiny_step = None
+    if world == 1 and not args.heads:
+        for name in (args.configs or []):
+            if name in configs:
+                continue
+            if name == "calib720":
+                sweep = calib_sweep(binding, dev, stream, pk, args.sweep_inputs)
+                configs[name] = sweep
+            else:
+                res, st = attention_config(binding, name, dev, pk, reps=max(6, args.steps // 2),
+                                           with_library=name != "tiny")
+                configs[name] = res
+                if name == "tiny":
+                    tiny_step = st
+                del st
+            torch.cuda.empty_cache()
+        if not args.no_calib:
+            calib = calibration_kernels(binding, wl, q, k, dev, stream, pk)
+        if args.fp8_probe:
+            fp8 = {name: fp8_probe(binding, name, n_in, dev, stream) for name, n_in in (("tiny", 8), ("wan480", 4))}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
@@ -587,6 +863,8 @@ def run_ours(args, world, rank, local):
                                                 args.cpu_seconds, np.random.default_rng(5))
         cpu = {"value": f / s / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{rows} query rows of one block-sparse head, fp64 plain-C oracle, {s:.1f} s"}
+        if tiny_step is not None:
+            cpu["tiny_full"] = tiny_oracle_full(tiny_step, configs["tiny"])
 
     if rank == 0:
         line = {
@@ -594,18 +872,51 @@ def run_ours(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "strong" if shard else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": arm_config(wl, heads, kept_frac, world, shard),
-            "gpu_launches": launches_per_step * args.steps,
+            "config": arm_config(wl, heads, step.kept_frac, world, shard),
+            "gpu_launches": step.launches * args.steps,
             "attn_ms": attn_ms,
-            "separate_calls": None if shard else {"sparse_ms": sparse_ms, "repeat_ms": repeat_ms,
-                                                  "sparse_tflops": f_sparse / (sparse_ms * 1e-3) / 1e12},
+            "separate_calls": separate,
             "dense_ms": dense_ms, "dense_tflops": f_dense / (dense_ms * 1e-3) / 1e12,
             "speedup_vs_dense": dense_ms / ms_step,
-            "library_dense": library_dense,
-            "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "calibration": calib,
+            "library_dense": lib_dense,
+            "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
+            "configs": configs, "calibration": calib, "fp8_probe": fp8,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
+
+
+def tiny_oracle_full(step, gpu_summary):
+    """The oracle's whole tiny pipeline, timed on the host cores: calibration
+    energies of the 8 inputs, greedy selection, aggregation, skip list, and the
+    masked attention of the held-out input. Reported beside it: the aggregated
+    cells where the oracle's mask and the GPU's differ (a selection whose cut
+    lies within the energy error of eps can go either way), and the largest
+    error of the GPU's output against the oracle's attention over the GPU's
+    own calibrated mask (the parity rule for the attention)."""
+    import oracle
+    wl = step.wl
+    threads = os.cpu_count() or 1
+    n_cal, eps = synth.CALIBRATION["tiny"]
+    t0 = time.perf_counter()
+    masks = []
+    for p in range(n_cal):
+        qc, kc, _ = synth.qkv(wl, p, with_v=False)
+        E = oracle.block_energy(synth.bf16_bits(qc), synth.bf16_bits(kc), threads=threads)
+        m, _ = oracle.select(E, eps)
+        masks.append(m)
+    agg, _ = oracle.aggregate(np.stack(masks), 0.5)
+    oracle.mask_to_csr(agg)
+    qb, kb, vb = (synth.bf16_bits(t) for t in (step.q, step.k, step.v))
+    oracle.masked_attention(qb, kb, vb, agg, threads=threads)
+    secs = time.perf_counter() - t0
+    o_ref, _ = oracle.masked_attention(qb, kb, vb, step.masks, threads=threads)
+    o_gpu = step.o.float().cpu().numpy().astype(np.float64)
+    err = float(np.max(np.abs(o_gpu - o_ref)))
+    return {"seconds": secs, "cores": threads, "what": "calibration of 8 inputs + selection + aggregation + "
+            "attention of the held-out input, fp64 plain C",
+            "max_abs_output_error_gpu_vs_oracle": err, "tolerance": 1e-2 * float(np.max(np.abs(o_ref))) + 1e-3,
+            "mask_cells_differing_from_gpu": int(np.sum(agg != step.masks))}
 
 
 def main():
@@ -622,10 +933,15 @@ def main():
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N>1: a replica of the call per rank (weak scaling) or one call split by heads (strong)")
     ap.add_argument("--no-calib", action="store_true")
+    ap.add_argument("--configs", default="tiny,wan480,mochi480,calib720",
+                    help="other workloads reported under 'configs' (comma-separated; 'none' for none)")
+    ap.add_argument("--sweep-inputs", type=int, default=64, help="calibration inputs of the sweep workload")
+    ap.add_argument("--no-fp8-probe", dest="fp8_probe", action="store_false")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="dram bytes per launch of the sparse kernel from an ncu capture")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.configs = [] if args.configs in ("", "none") else [c.strip() for c in args.configs.split(",")]
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -730,7 +730,7 @@ int calibatt_accumulate_masks(const uint8_t* mask, int64_t cells, uint16_t* coun
 
 size_t calibatt_aggregate_workspace_size(int heads, int nb) {
   if (heads < 1 || nb < 1) return 0;
-  const size_t bytes = static_cast<size_t>(heads) * nb * sizeof(int32_t);
+  const size_t bytes = static_cast<size_t>(aggregate_scratch_ints(static_cast<int64_t>(heads) * nb)) * sizeof(int32_t);
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 

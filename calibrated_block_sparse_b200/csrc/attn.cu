@@ -71,6 +71,7 @@ struct AttnLayout {
   static constexpr int kDynSmem = kBytes + 1024;  // + alignment slack
 };
 
+template <bool SW>  // SW: the polling wait form of short (test) wait limits
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qb,
                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t stage = 0, phase = 0, n_q[2] = {0, 0};
       bool ok = true;
       auto load_tile = [&](const CUtensorMap* map, int blk, int head) -> bool {
-        if (!mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns)) return false;
+        if (!mbar_wait<SW>(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns)) return false;
         uint8_t* dst = smem + L::kRingOff + stage * kTile;
         mbar_arrive_expect_tx(&bar.ring_full[stage], kTile);
         tma_load_3d(dst, map, &bar.ring_full[stage], 0, blk * 128, head);
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       auto emit_s = [&](int s) -> bool {
         Cursor& c = cur[s];
         if (c.j == 0) {
-          if (!mbar_wait(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) return false;
+          if (!mbar_wait<SW>(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) return false;
           uint8_t* dst = smem + L::kQOff + s * kTile;
           const CUtensorMap* qmap = c.u.rep ? &tm_qb : &tm_q;
           mbar_arrive_expect_tx(&bar.q_full[s], kTile);
@@ -197,9 +198,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       auto issue_s = [&](int s) -> bool {
         Cursor& c = cur[s];
         if (c.j == 0) {
-          if (!mbar_wait(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status, p.wait_limit_ns)) return false;
+          if (!mbar_wait<SW>(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status, p.wait_limit_ns)) return false;
         }
-        if (!mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status, p.wait_limit_ns)) return false;
+        if (!mbar_wait<SW>(&bar.ring_full[stage], phase, abort_flag, p.status, p.wait_limit_ns)) return false;
         tc_fence_after();
         const uint64_t qd = qdesc0 + s * (kTile >> 4), kd = kdesc0 + stage * (kTile >> 4);
 #pragma unroll
@@ -220,8 +221,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int s = 0; s < 2 && ok; ++s) {
           if (!cur[s].valid) continue;
           // O += P V for the current block of slot s (P read from tensor memory)
-          if (!(ok = mbar_wait(&bar.p_full[s], n_pv[s] & 1, abort_flag, p.status, p.wait_limit_ns))) break;
-          if (!(ok = mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status, p.wait_limit_ns))) break;
+          if (!(ok = mbar_wait<SW>(&bar.p_full[s], n_pv[s] & 1, abort_flag, p.status, p.wait_limit_ns))) break;
+          if (!(ok = mbar_wait<SW>(&bar.ring_full[stage], phase, abort_flag, p.status, p.wait_limit_ns))) break;
           tc_fence_after();
           const uint64_t vd = vdesc0 + stage * (kTile >> 4);
 #pragma unroll
@@ -257,7 +258,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t n_sfull = 0, n_ofull = 0;
     bool ok = true;  // warp-uniform
     auto wait_warp = [&](uint64_t* b, uint32_t parity) -> bool {
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, p.status, p.wait_limit_ns));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait<SW>(b, parity, abort_flag, p.status, p.wait_limit_ns));
       return ok;
     };
 
@@ -392,23 +393,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 int launch_attn(const CUtensorMap& mq, const CUtensorMap& mqb, const CUtensorMap& mk, const CUtensorMap& mv,
                 const KernelParams& p, cudaStream_t stream) {
   static_assert(AttnLayout::kDynSmem <= 232448, "shared memory budget");
-  static PerDeviceOnce smem_once;
-  int rc = set_max_smem_once(reinterpret_cast<const void*>(attn_kernel), AttnLayout::kDynSmem, smem_once);
+  const bool short_waits = p.wait_limit_ns < kShortWaitNs;
+  const void* fn = short_waits ? reinterpret_cast<const void*>(attn_kernel<true>)
+                               : reinterpret_cast<const void*>(attn_kernel<false>);
+  static PerDeviceOnce smem_once[2];
+  int rc = set_max_smem_once(fn, AttnLayout::kDynSmem, smem_once[short_waits ? 1 : 0]);
   if (rc != CALIBATT_OK) return rc;
   // the register split needs the allotment it was sized for (a property of
-  // the compiled kernel, the same on every device)
+  // the compiled kernels, the same on every device)
   static std::once_flag regs_once;
   static int launch_regs = 0;
   std::call_once(regs_once, [] {
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_kernel) == cudaSuccess) launch_regs = fa.numRegs;
+    cudaFuncAttributes fa, fb;
+    if (cudaFuncGetAttributes(&fa, attn_kernel<false>) == cudaSuccess &&
+        cudaFuncGetAttributes(&fb, attn_kernel<true>) == cudaSuccess)
+      launch_regs = fa.numRegs < fb.numRegs ? fa.numRegs : fb.numRegs;
   });
   if (launch_regs * kAttnThreads < 256 * kSoftmaxRegs + 128 * kControlRegs) return CALIBATT_ERR_CUDA;
   if (p.n_units <= 0) return CALIBATT_OK;
   int grid = (p.n_units + 1) / 2;
   const int sms = sm_count();
   if (grid > sms) grid = sms;
-  attn_kernel<<<grid, kAttnThreads, AttnLayout::kDynSmem, stream>>>(mq, mqb, mk, mv, p);
+  if (short_waits)
+    attn_kernel<true><<<grid, kAttnThreads, AttnLayout::kDynSmem, stream>>>(mq, mqb, mk, mv, p);
+  else
+    attn_kernel<false><<<grid, kAttnThreads, AttnLayout::kDynSmem, stream>>>(mq, mqb, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
 }
 

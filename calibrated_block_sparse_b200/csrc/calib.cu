@@ -16,21 +16,21 @@ namespace calibatt {
 
 
 // ------------------------------------------------------------------ selection
-// One warp per block-row of energies, four rows per CTA, each warp with its
-// own 8 KB histogram; no block barriers. PER (columns per lane, >= nb / 32)
+// One warp per block-row of energies, four rows per CTA, each warp with 128
+// bytes of shared scratch; no block barriers. PER (columns per lane, >= nb / 32)
 // sizes the per-lane register arrays. Lanes read and write the row's columns
 // interleaved (column lane + 32 i), so every access is coalesced.
 template <int PER>
 __global__ void __launch_bounds__(128) select_kernel(const float* __restrict__ energy, int64_t rows, int nb,
                                                      long long eps_fx, uint8_t* mask, int32_t* kept,
                                                      uint16_t* counts, uint8_t* tie, long long tie_fx) {
-  __shared__ __align__(16) unsigned long long hist[4][kSelectBuckets];
+  __shared__ __align__(16) float scratch[4][kSelectScratchBytes / 4];
   const int w = threadIdx.x >> 5;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + w;
   if (row >= rows) return;
   SelectOut out{mask ? mask + row * nb : nullptr, kept ? kept + row : nullptr, counts ? counts + row * nb : nullptr,
                 tie ? tie + row : nullptr};
-  warp_select<PER>(energy + row * nb, nb, eps_fx, tie_fx, hist[w], out);
+  warp_select<PER>(energy + row * nb, nb, eps_fx, tie_fx, scratch[w], out);
 }
 
 // ------------------------------------------------------------------ accumulation
@@ -43,109 +43,90 @@ __global__ void accumulate_kernel(const uint8_t* __restrict__ mask, int64_t cell
 }
 
 // ------------------------------------------------------------------ aggregation
-// Pass 1: one warp per (head, block-row): binarise counts >= threshold, write
-// the mask row and the row's kept count.
-__global__ void binarize_kernel(const uint16_t* __restrict__ counts, int64_t rows, int nb, int threshold,
-                                uint8_t* mask, int32_t* row_cnt) {
-  const int64_t row = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const uint16_t* src = counts + row * nb;
-  uint8_t* dst = mask + row * nb;
+// Two launches over CTAs of kAggRows block-rows (one warp per row):
+//  1. binarize: counts >= threshold -> mask row, the row's kept count, and
+//     the CTA's total;
+//  2. compact: each CTA adds up the totals of the CTAs before it (all final
+//     once the first launch is done: no cross-CTA waiting), scans its own
+//     rows' counts into row_ptr (global offsets), and writes each row's kept
+//     columns in ascending order. The last CTA writes the grand total.
+// Scratch: row_cnt[rows] then cta_sum[ceil(rows / kAggRows)].
+constexpr int kAggRows = 32;  // = warps per CTA = lanes of a warp (partials are read one per lane)
+
+__global__ void __launch_bounds__(kAggRows * 32) binarize_kernel(const uint16_t* __restrict__ counts, int64_t rows,
+                                                                 int nb, int threshold, uint8_t* mask,
+                                                                 int32_t* row_cnt, int32_t* cta_sum) {
+  __shared__ int wsum[kAggRows];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kAggRows + w;
   int cnt = 0;
-  for (int c = lane; c < nb; c += 32) {
-    const uint8_t k = src[c] >= threshold ? 1 : 0;
-    dst[c] = k;
-    cnt += k;
+  if (row < rows) {
+    const uint16_t* src = counts + row * nb;
+    uint8_t* dst = mask + row * nb;
+#pragma unroll 4
+    for (int c = lane; c < nb; c += 32) {
+      const uint8_t k = src[c] >= threshold ? 1 : 0;
+      dst[c] = k;
+      cnt += k;
+    }
+    cnt = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
+    if (lane == 0) row_cnt[row] = cnt;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) row_cnt[row] = cnt;
+  if (lane == 0) wsum[w] = cnt;
+  __syncthreads();
+  if (w == 0) {
+    const int t = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(wsum[lane])));
+    if (lane == 0) cta_sum[blockIdx.x] = t;
+  }
 }
 
-// Pass 2: a single CTA turns the row counts into the exclusive prefix row_ptr
-// (global offsets) and the total. The counts are taken in tiles of
-// kScanTile rows staged in shared memory (coalesced); each thread scans a
-// contiguous run of its tile, one block-wide scan of the 1024 run totals
-// joins them, and a carry crosses tiles. One padding word per 32 keeps the
-// threads' runs on distinct banks.
-constexpr int kScanThreads = 1024;
-constexpr int kScanTile = 16384;  // rows per tile
-constexpr int kScanSmem = (kScanTile + kScanTile / 32) * 4;
-
-__device__ __forceinline__ int scan_pad(int i) { return i + (i >> 5); }
-
-__global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t* __restrict__ row_cnt, int64_t rows,
-                                                            int32_t* row_ptr, int64_t nnz_cap, int64_t* nnz_out,
-                                                            int* status) {
-  extern __shared__ int32_t tile[];
-  __shared__ long long warp_tot[32];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  constexpr int kRun = kScanTile / kScanThreads;
-  long long carry = 0;
-  for (int64_t base = 0; base < rows; base += kScanTile) {
-    const int n = static_cast<int>(rows - base < kScanTile ? rows - base : kScanTile);
-    for (int i = tid; i < n; i += kScanThreads) tile[scan_pad(i)] = row_cnt[base + i];
-    __syncthreads();
-    long long run = 0;
+__global__ void __launch_bounds__(kAggRows * 32) compact_kernel(const uint8_t* __restrict__ mask, int64_t rows,
+                                                                int nb, const int32_t* __restrict__ row_cnt,
+                                                                const int32_t* __restrict__ cta_sum,
+                                                                int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap,
+                                                                int64_t* nnz_out, int* status) {
+  __shared__ long long wpart[kAggRows];
+  __shared__ int wcnt[kAggRows];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the kept blocks of every earlier CTA
+  long long before = 0;
+  for (int64_t i = threadIdx.x; i < blockIdx.x; i += blockDim.x) before += cta_sum[i];
 #pragma unroll
-    for (int k = 0; k < kRun; ++k) {
-      const int i = tid * kRun + k;
-      run += i < n ? tile[scan_pad(i)] : 0;
-    }
-    long long incl = run;
+  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kAggRows + w;
+  const int cnt = row < rows ? row_cnt[row] : 0;
+  if (lane == 0) {
+    wpart[w] = before;
+    wcnt[w] = cnt;
+  }
+  __syncthreads();
+  // lane i of every warp takes warp i's partials
+  long long base = wpart[lane];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    if (lane == 31) warp_tot[w] = incl;
-    __syncthreads();
-    long long wbefore = 0, all = 0;
-    for (int ww = 0; ww < 32; ++ww) {
-      const long long t = warp_tot[ww];
-      wbefore += ww < w ? t : 0;
-      all += t;
-    }
-    long long pos = carry + wbefore + incl - run;  // exclusive prefix of this thread's run
-#pragma unroll
-    for (int k = 0; k < kRun; ++k) {
-      const int i = tid * kRun + k;
-      if (i < n) {
-        const int32_t v = tile[scan_pad(i)];
-        tile[scan_pad(i)] = static_cast<int32_t>(pos);
-        pos += v;
+  for (int o = 16; o > 0; o >>= 1) base += __shfl_xor_sync(0xffffffffu, base, o);
+  const unsigned cw = static_cast<unsigned>(wcnt[lane]);
+  const long long mine = __reduce_add_sync(0xffffffffu, lane < w ? cw : 0u);
+  const long long total = __reduce_add_sync(0xffffffffu, cw);
+  long long pos = base + mine;  // this row's first entry
+  if (row < rows) {
+    if (lane == 0) row_ptr[row] = static_cast<int32_t>(pos);
+    const uint8_t* src = mask + row * nb;
+    for (int c0 = 0; c0 < nb; c0 += 32) {
+      const int c = c0 + lane;
+      const bool k = c < nb && src[c];
+      const uint32_t bal = __ballot_sync(0xffffffffu, k);
+      if (k) {
+        const int64_t at = pos + __popc(bal & ((1u << lane) - 1u));
+        if (at < nnz_cap) col_idx[at] = c;
       }
+      pos += __popc(bal);
     }
-    __syncthreads();
-    for (int i = tid; i < n; i += kScanThreads) row_ptr[base + i] = tile[scan_pad(i)];
-    carry += all;
-    __syncthreads();  // the tile and warp totals are reused
   }
-  if (tid == 0) {
-    row_ptr[rows] = static_cast<int32_t>(carry);
-    *nnz_out = carry;
-    if (carry > nnz_cap) record_error(status, CALIBATT_ERR_CAPACITY);
-  }
-}
-
-// Pass 3: one warp per row writes the kept columns in ascending order.
-__global__ void compact_kernel(const uint8_t* __restrict__ mask, int64_t rows, int nb,
-                               const int32_t* __restrict__ row_ptr, int32_t* col_idx, int64_t nnz_cap) {
-  const int64_t row = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const uint8_t* src = mask + row * nb;
-  int64_t pos = row_ptr[row];
-  for (int c0 = 0; c0 < nb; c0 += 32) {
-    const int c = c0 + lane;
-    const bool k = c < nb && src[c];
-    const uint32_t bal = __ballot_sync(0xffffffffu, k);
-    if (k) {
-      const int64_t at = pos + __popc(bal & ((1u << lane) - 1u));
-      if (at < nnz_cap) col_idx[at] = c;
-    }
-    pos += __popc(bal);
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
+    const long long grand = base + total;
+    row_ptr[rows] = static_cast<int32_t>(grand);
+    *nnz_out = grand;
+    if (grand > nnz_cap) record_error(status, CALIBATT_ERR_CAPACITY);
   }
 }
 
@@ -206,17 +187,18 @@ int launch_accumulate(const uint8_t* mask, int64_t cells, uint16_t* counts, cuda
 }
 
 int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold, uint8_t* mask, int32_t* row_ptr,
-                     int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* row_cnt, int* status,
+                     int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* scratch, int* status,
                      cudaStream_t stream) {
-  const unsigned warps_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
-  static PerDeviceOnce scan_once;
-  const int rc = set_max_smem_once(reinterpret_cast<const void*>(scan_kernel), kScanSmem, scan_once);
-  if (rc != CALIBATT_OK) return rc;
-  binarize_kernel<<<warps_blocks, 256, 0, stream>>>(counts, rows, nb, threshold, mask, row_cnt);
-  scan_kernel<<<1, kScanThreads, kScanSmem, stream>>>(row_cnt, rows, row_ptr, nnz_cap, nnz, status);
-  compact_kernel<<<warps_blocks, 256, 0, stream>>>(mask, rows, nb, row_ptr, col_idx, nnz_cap);
+  const unsigned ctas = static_cast<unsigned>((rows + kAggRows - 1) / kAggRows);
+  int32_t* row_cnt = scratch;
+  int32_t* cta_sum = scratch + rows;
+  binarize_kernel<<<ctas, kAggRows * 32, 0, stream>>>(counts, rows, nb, threshold, mask, row_cnt, cta_sum);
+  compact_kernel<<<ctas, kAggRows * 32, 0, stream>>>(mask, rows, nb, row_cnt, cta_sum, row_ptr, col_idx, nnz_cap, nnz,
+                                                     status);
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
 }
+
+int64_t aggregate_scratch_ints(int64_t rows) { return rows + (rows + kAggRows - 1) / kAggRows; }
 
 int launch_gather(const void* q, int n, int heads, const int32_t* rep_heads, int n_rep, int H, int W, int k_anchor,
                   const AnchorTable& tab, void* out, int* status, cudaStream_t stream) {

@@ -79,9 +79,12 @@ long long eps_to_fixed(double eps);
 int launch_select(const float* energy, int64_t rows, int nb, long long eps_fx, uint8_t* mask, int32_t* kept,
                   uint16_t* counts, uint8_t* tie, long long tie_fx, cudaStream_t stream);
 int launch_accumulate(const uint8_t* mask, int64_t cells, uint16_t* counts, cudaStream_t stream);
+// scratch: aggregate_scratch_ints(rows) int32 (per-row kept counts, then one
+// total per CTA of rows), every entry rewritten by each call
 int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold, uint8_t* mask, int32_t* row_ptr,
-                     int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* row_cnt, int* status,
+                     int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* scratch, int* status,
                      cudaStream_t stream);
+int64_t aggregate_scratch_ints(int64_t rows);
 int launch_spatial_score(const float* pix, int heads, int frames, int H, int nb, const RowAnchorTable& tab,
                          float gamma, float* score, uint8_t* flag, cudaStream_t stream);
 int launch_gather(const void* q, int n, int heads, const int32_t* rep_heads, int n_rep, int H, int W, int k_anchor,

@@ -18,9 +18,11 @@
 
 namespace calibatt {
 
-// One int32 per (head, block-row): at most CALIBATT_NOALLOC_MAX_ROWS rows
-// (1 MiB). Every GPU that loads the library holds this array until exit.
-static __device__ __align__(256) int32_t g_noalloc_row_cnt[CALIBATT_NOALLOC_MAX_ROWS];
+// One int32 per (head, block-row), at most CALIBATT_NOALLOC_MAX_ROWS rows,
+// then one per group of 32 rows: 1 MiB + 32 KiB. Every GPU that loads the
+// library holds this array until exit.
+constexpr int64_t kNoallocScratchInts = CALIBATT_NOALLOC_MAX_ROWS + CALIBATT_NOALLOC_MAX_ROWS / 32;
+static __device__ __align__(256) int32_t g_noalloc_row_cnt[kNoallocScratchInts];
 
 namespace {
 
@@ -58,13 +60,14 @@ extern "C" int calibatt_aggregate_masks_noalloc(const uint16_t* counts, int n_in
   if ((reinterpret_cast<uintptr_t>(counts) & 1u) || (reinterpret_cast<uintptr_t>(row_ptr) & 3u) ||
       (col_idx && (reinterpret_cast<uintptr_t>(col_idx) & 3u)) || (reinterpret_cast<uintptr_t>(nnz) & 7u))
     return CALIBATT_ERR_ALIGN;
+  if (aggregate_scratch_ints(rows) > kNoallocScratchInts) return CALIBATT_ERR_ARG;
   int32_t* scratch = noalloc_scratch();
   int* status = status_word();
   if (!scratch || !status) return CALIBATT_ERR_CUDA;
   int32_t thr = 0;
   calibatt_rho_threshold(n_inputs, rho, &thr);
-  // The binarize pass writes every one of the `rows` counts before the scan
-  // reads them, so the array needs no clearing between calls.
+  // The first pass writes every per-row count and per-group total that the
+  // second reads, so the array needs no clearing between calls.
   return launch_aggregate(counts, rows, nb, thr, mask, row_ptr, col_idx, nnz_cap, nnz, scratch, status,
                           reinterpret_cast<cudaStream_t>(stream));
 }

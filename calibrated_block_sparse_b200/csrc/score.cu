@@ -70,7 +70,14 @@ struct ScoreLayout {
   static constexpr int kDynSmem = kBytes + 1024;  // + alignment slack
 };
 
-template <int MODE>
+// The fused selection: one call per finished row, kept out of line so that
+// its registers do not weigh on the kernel's main loop.
+__device__ __noinline__ void warp_select_row1024(const float* E, int nb, long long eps_fx, long long tie_fx,
+                                                 float* scratch, SelectOut out) {
+  warp_select<32>(E, nb, eps_fx, tie_fx, scratch, out);
+}
+
+template <int MODE, bool SW>  // SW: the polling wait form of short (test) wait limits
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ KernelParams p) {
@@ -124,14 +131,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         Cursor& c = cur[s];
         if (!c.valid) continue;
         if (c.j == 0) {
-          if (!(ok = mbar_wait(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns))) break;
+          if (!(ok = mbar_wait<SW>(&bar.q_empty[s], (n_q[s] & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns))) break;
           uint8_t* dst = smem + L::kQOff + s * kTile;
           mbar_arrive_expect_tx(&bar.q_full[s], kTile);
           tma_load_3d(dst, &tm_q, &bar.q_full[s], 0, c.u.r * 128, c.u.hq);
           tma_load_3d(dst + kHalf, &tm_q, &bar.q_full[s], 64, c.u.r * 128, c.u.hq);
           ++n_q[s];
         }
-        if (!(ok = mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns))) break;
+        if (!(ok = mbar_wait<SW>(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns))) break;
         bar.first[stage] = c.j == 0;
         bar.last[stage] = c.j == c.u.nnz - 1;
         bar.slot[stage] = s;
@@ -147,7 +154,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       }
     }
     bool marker = false;
-    if (ok && mbar_wait(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
+    if (ok && mbar_wait<SW>(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
       bar.end = 1;
       bar.slot[stage] = 2;  // end marker
       mbar_arrive(&bar.ring_full[stage]);
@@ -180,7 +187,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const uint64_t qdesc0 = desc_k_base(sbase + L::kQOff);
     const uint64_t kdesc0 = desc_k_base(sbase + L::kRingOff);
     while (true) {
-      if (!mbar_wait(&bar.ring_full[stage], phase, abort_flag, p.status, p.wait_limit_ns)) break;
+      if (!mbar_wait<SW>(&bar.ring_full[stage], phase, abort_flag, p.status, p.wait_limit_ns)) break;
       // read every word of the stage now: once ring_empty is committed below,
       // the producer may reuse the stage and rewrite them for its next tile
       const uint32_t s = *reinterpret_cast<volatile uint32_t*>(&bar.slot[stage]);
@@ -188,10 +195,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       const bool first = *reinterpret_cast<volatile uint32_t*>(&bar.first[stage]) != 0;
       const bool last = *reinterpret_cast<volatile uint32_t*>(&bar.last[stage]) != 0;
       if (first) {
-        if (!mbar_wait(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status, p.wait_limit_ns)) break;
+        if (!mbar_wait<SW>(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status, p.wait_limit_ns)) break;
       }
       const int buf = n_s[s] & 1;
-      if (!mbar_wait(&bar.s_empty[s][buf], ((n_s[s] >> 1) & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) break;
+      if (!mbar_wait<SW>(&bar.s_empty[s][buf], ((n_s[s] >> 1) & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + (2 * s + buf) * 128;
       const uint64_t qd = qdesc0 + s * (kTile >> 4), kd = kdesc0 + stage * (kTile >> 4);
@@ -262,7 +269,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       for (int j = 0; j < u.nnz; ++j) {
         const int buf = n_sfull & 1;
         float acc = 0.f;
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_full[s][buf], (n_sfull >> 1) & 1, abort_flag,
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait<SW>(&bar.s_full[s][buf], (n_sfull >> 1) & 1, abort_flag,
                                                        p.status, p.wait_limit_ns));
         if (ok) {
           ++n_sfull;
@@ -365,14 +372,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
         if (p.fuse_select) {
           // the finished row is selected by the warpgroup's first warp
-          // (its 8 KB histogram behind the row in the slot's scratch)
+          // (its candidate scratch behind the row in the slot's scratch)
           named_bar_sync(1 + s, 128);
           if (wl == 0) {
             const int64_t urow = erow / p.nbk;
             SelectOut out{p.mask ? p.mask + erow : nullptr, p.kept ? p.kept + urow : nullptr,
                           p.counts ? p.counts + erow : nullptr, p.tie ? p.tie + urow : nullptr};
             if (!ok) out = SelectOut{nullptr, nullptr, nullptr, nullptr};
-            warp_select<32>(part, p.nbk, p.eps_fx, p.tie_fx, reinterpret_cast<unsigned long long*>(part + 1024), out);
+            warp_select_row1024(part, p.nbk, p.eps_fx, p.tie_fx, part + 1024, out);
           }
         }
         named_bar_sync(1 + s, 128);
@@ -395,11 +402,17 @@ int launch_mode(const CUtensorMap& mq, const CUtensorMap& mk, const KernelParams
   using L = ScoreLayout<MODE>;
   static_assert(L::kDynSmem <= 232448, "shared memory budget");
   static_assert(kEnergyScratch >= 4096 + kSelectScratchBytes, "selection scratch behind the energy row");
-  static PerDeviceOnce smem_once;
-  const int rc = set_max_smem_once(reinterpret_cast<const void*>(score_kernel<MODE>), L::kDynSmem, smem_once);
+  const bool short_waits = p.wait_limit_ns < kShortWaitNs;
+  const void* fn = short_waits ? reinterpret_cast<const void*>(score_kernel<MODE, true>)
+                               : reinterpret_cast<const void*>(score_kernel<MODE, false>);
+  static PerDeviceOnce smem_once[2];
+  const int rc = set_max_smem_once(fn, L::kDynSmem, smem_once[short_waits ? 1 : 0]);
   if (rc != CALIBATT_OK) return rc;
   if (p.n_units <= 0) return CALIBATT_OK;
-  score_kernel<MODE><<<score_grid(p.n_units), kScoreThreads, L::kDynSmem, stream>>>(mq, mk, p);
+  if (short_waits)
+    score_kernel<MODE, true><<<score_grid(p.n_units), kScoreThreads, L::kDynSmem, stream>>>(mq, mk, p);
+  else
+    score_kernel<MODE, false><<<score_grid(p.n_units), kScoreThreads, L::kDynSmem, stream>>>(mq, mk, p);
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
 }
 
