@@ -88,6 +88,14 @@ def load(build_if_missing: bool = False):
             "calibatt_mixed_attn_fwd": (i32, [P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, i64, P, i32, P, i32,
                                               P, P, P, sz, P]),
             "calibatt_spatial_score": (i32, [P, i32, i32, i32, i32, i32, f32, P, P, P]),
+            "calibatt_balance_mixed_plan": (i32, [P, i32, P, i32, i32, P, i32, i32, i32, i32, i32]),
+            "calibatt_mixed_masked_attn_fwd": (i32, [P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, i64, P, i32,
+                                                     P, P, i64, P, i32, P, P, P, sz, P]),
+            "calibatt_anchor_energy_workspace_size": (sz, [i32, i32, i32, i32, i32, i32]),
+            "calibatt_anchor_block_energy": (i32, [P, P, i32, i32, i32, i32, i32, i32, f32, P, i32, P, sz, P, i32,
+                                                   f64, P, P, P, P, f64, P]),
+            "calibatt_aggregate_rows_workspace_size": (sz, [i64]),
+            "calibatt_aggregate_mask_rows": (i32, [P, i32, i64, i32, f64, P, P, P, i64, P, P, sz, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -317,6 +325,52 @@ def mixed_attn_fwd(q, k, v, F, H, W, row_ptr, col_idx, rep_heads, work_list, k_a
     return o, lse
 
 
+def anchor_blocks(F, W, k_anchor=5) -> int:
+    """Blocks of 128 packed anchor queries of one repeated head."""
+    return -(-F * k_anchor * W // BLOCK)
+
+
+def balance_mixed_plan(work_list: np.ndarray, row_ptr: np.ndarray, heads: int, nb: int, row_ptr_b, n_rep: int,
+                       F: int, W: int, k_anchor: int = 5, n_slots: int = 0) -> np.ndarray:
+    """calibatt_balance_mixed_plan on a copy of a host work list (anchor units
+    costed by the anchor skip list row_ptr_b, host int32)."""
+    w = np.array(work_list, dtype=np.int32, copy=True)
+    rp = np.ascontiguousarray(row_ptr, np.int32)
+    rpb = None if row_ptr_b is None else np.ascontiguousarray(row_ptr_b, np.int32)
+    _check(load().calibatt_balance_mixed_plan(_ptr(w), int(w.size), _ptr(rp), int(heads), int(nb), _ptr(rpb),
+                                              int(n_rep), int(F), int(W), int(k_anchor), int(n_slots)),
+           "calibatt_balance_mixed_plan")
+    return w
+
+
+def mixed_masked_attn_fwd(q, k, v, F, H, W, row_ptr, col_idx, rep_heads, row_ptr_b, col_idx_b, work_list, k_anchor=5,
+                          o=None, lse=None, ws=None, scale=None, want_lse=True, stream=None):
+    """calibatt_mixed_masked_attn_fwd: block-sparse heads over their skip lists,
+    repeated heads' anchor rows over their own anchor skip list; returns (o, lse)."""
+    heads, n = _bhnd(q)
+    _bhnd(k, "k")
+    _bhnd(v, "v")
+    for t, name in ((row_ptr, "row_ptr"), (col_idx, "col_idx"), (rep_heads, "rep_heads"), (row_ptr_b, "row_ptr_b"),
+                    (col_idx_b, "col_idx_b"), (work_list, "work_list")):
+        _cuda_tensor(t, torch.int32, name)
+    n_rep = rep_heads.numel()
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((heads, n), dtype=torch.float32, device=q.device)
+    if ws is None and n_rep > 0:
+        ws = torch.empty(repeat_workspace_size(n_rep, F, H, W, k_anchor), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = load().calibatt_mixed_masked_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), heads, F, H, W, HEAD_DIM, k_anchor, scale, _ptr(row_ptr),
+        _ptr(col_idx) if col_idx.numel() else None, col_idx.numel(), _ptr(rep_heads) if n_rep else None, n_rep,
+        _ptr(row_ptr_b) if row_ptr_b.numel() else None, _ptr(col_idx_b) if col_idx_b.numel() else None,
+        col_idx_b.numel(), _ptr(work_list) if work_list.numel() else None, work_list.numel(), _ptr(o), _ptr(lse),
+        _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream))
+    _check(rc, "calibatt_mixed_masked_attn_fwd")
+    return o, lse
+
+
 def mixed_attn_fwd_host(q_host, k_host, v_host, o_host, F, H, W, row_ptr_host, row_ptr, col_idx, rep_heads,
                         q_dev, k_dev, v_dev, o_dev, lse_host=None, lse_dev=None, ws=None, heads_per_chunk=2,
                         k_anchor=5, scale=None, stream=None):
@@ -457,6 +511,65 @@ def block_energy_1pass(q, k, eps=None, energy=True, mask=None, kept=None, counts
                                             int(pix_W or 0), _stream(stream))
     _check(rc, "calibatt_block_energy_1pass")
     return (e, mask, kept, counts, pix, tie) if want_tie else (e, mask, kept, counts, pix)
+
+
+def anchor_block_energy(q, k, F, H, W, rep_heads, k_anchor=5, eps=None, energy=True, mask=None, kept=None,
+                        counts=None, ws=None, scale=None, stream=None, tie=None, tie_window=TIE_WINDOW):
+    """Block energies of the repeated heads' anchor queries, [n_rep][nbq][nb]
+    (with eps, the fused greedy selection too). Returns (energy or None, mask,
+    kept, counts), plus the tie flags when tie is True or a tensor."""
+    heads, n = _bhnd(q)
+    if n != F * H * W:
+        raise ValueError(f"n = {n} is not F*H*W = {F * H * W}")
+    _cuda_tensor(rep_heads, torch.int32, "rep_heads")
+    n_rep = rep_heads.numel()
+    nb = (n + BLOCK - 1) // BLOCK
+    nbq = anchor_blocks(F, W, k_anchor)
+    dev = q.device
+    lib = load()
+    if ws is None:
+        ws = torch.empty(lib.calibatt_anchor_energy_workspace_size(heads, n_rep, F, H, W, k_anchor),
+                         dtype=torch.uint8, device=dev)
+    e = torch.empty((n_rep, nbq, nb), dtype=torch.float32, device=dev) if energy is True else (
+        energy if isinstance(energy, torch.Tensor) else None)
+    fuse = eps is not None
+    if fuse and mask is None and kept is None and counts is None:
+        mask = torch.empty((n_rep, nbq, nb), dtype=torch.uint8, device=dev)
+        kept = torch.empty((n_rep, nbq), dtype=torch.int32, device=dev)
+    want_tie = tie is not None and tie is not False
+    tie = _tie_out(tie, (n_rep, nbq), dev)
+    scale = 1.0 / math.sqrt(HEAD_DIM) if scale is None else float(scale)
+    rc = lib.calibatt_anchor_block_energy(_ptr(q), _ptr(k), heads, F, H, W, HEAD_DIM, k_anchor, scale,
+                                          _ptr(rep_heads), n_rep, _ptr(ws), ws.numel(), _ptr(e), 1 if fuse else 0,
+                                          float(eps) if fuse else 0.0, _ptr(mask), _ptr(kept), _ptr(counts),
+                                          _ptr(tie), float(tie_window), _stream(stream))
+    _check(rc, "calibatt_anchor_block_energy")
+    return (e, mask, kept, counts, tie) if want_tie else (e, mask, kept, counts)
+
+
+def aggregate_mask_rows(counts, n_inputs, rho=0.5, nnz_cap=None, ws=None, stream=None, trim=True):
+    """Binarise [rows][cols] counts at rho and build their CSR skip list;
+    returns (mask, row_ptr, col_idx, nnz)."""
+    _cuda_tensor(counts, torch.uint16, "counts")
+    cols = counts.shape[-1]
+    rows = counts.numel() // cols
+    dev = counts.device
+    if nnz_cap is None:
+        nnz_cap = rows * cols
+    mask = torch.empty(counts.shape, dtype=torch.uint8, device=dev)
+    row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(int(nnz_cap), 1), dtype=torch.int32, device=dev)
+    nnz = torch.zeros(1, dtype=torch.int64, device=dev)
+    lib = load()
+    if ws is None:
+        ws = torch.empty(lib.calibatt_aggregate_rows_workspace_size(rows), dtype=torch.uint8, device=dev)
+    rc = lib.calibatt_aggregate_mask_rows(_ptr(counts), int(n_inputs), rows, cols, float(rho), _ptr(mask),
+                                          _ptr(row_ptr), _ptr(col_idx), int(nnz_cap), _ptr(nnz), _ptr(ws), ws.numel(),
+                                          _stream(stream))
+    _check(rc, "calibatt_aggregate_mask_rows")
+    if trim:
+        col_idx = col_idx[:int(nnz.item())]
+    return mask, row_ptr, col_idx, nnz
 
 
 def select_mask(energy, eps, mask=True, kept=True, counts=None, stream=None, tie=None, tie_window=TIE_WINDOW):

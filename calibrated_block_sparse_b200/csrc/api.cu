@@ -286,8 +286,11 @@ int calibatt_build_mixed_plan(const int32_t* row_ptr, int heads, int nb, const u
   return CALIBATT_OK;
 }
 
-int calibatt_balance_plan(int32_t* work_list, int32_t n_work, const int32_t* row_ptr, int heads, int nb,
-                          int n_slots) {
+namespace {
+// calibatt_balance_plan with the anchor-query units' costs taken from their
+// own skip list (row_ptr_b [n_rep * nbq_b + 1]) when given.
+int balance_plan(int32_t* work_list, int32_t n_work, const int32_t* row_ptr, int heads, int nb,
+                 const int32_t* row_ptr_b, int64_t n_b_units, int n_slots) {
   if (!work_list || n_work < 0 || !row_ptr || heads < 1 || nb < 1) return CALIBATT_ERR_ARG;
   if (n_work == 0) return CALIBATT_OK;
   if (n_slots <= 0) {
@@ -304,6 +307,8 @@ int calibatt_balance_plan(int32_t* work_list, int32_t n_work, const int32_t* row
   const int64_t n_a = static_cast<int64_t>(heads) * nb;
   auto cost = [&](int32_t code) -> int64_t {
     if (code >= 0 && code < n_a) return static_cast<int64_t>(row_ptr[code + 1]) - row_ptr[code] + 2;
+    if (code >= n_a && row_ptr_b && code - n_a < n_b_units)  // anchor-query unit with its own skip list
+      return static_cast<int64_t>(row_ptr_b[code - n_a + 1]) - row_ptr_b[code - n_a] + 2;
     if (code >= n_a) return nb + 2;  // anchor-query unit: every key block
     return 2;
   };
@@ -325,6 +330,20 @@ int calibatt_balance_plan(int32_t* work_list, int32_t n_work, const int32_t* row
     }
   }
   return CALIBATT_OK;
+}
+}  // namespace
+
+int calibatt_balance_plan(int32_t* work_list, int32_t n_work, const int32_t* row_ptr, int heads, int nb,
+                          int n_slots) {
+  return balance_plan(work_list, n_work, row_ptr, heads, nb, nullptr, 0, n_slots);
+}
+
+int calibatt_balance_mixed_plan(int32_t* work_list, int32_t n_work, const int32_t* row_ptr, int heads, int nb,
+                                const int32_t* row_ptr_b, int n_rep, int frames, int W, int k_anchor, int n_slots) {
+  if (n_rep < 0 || frames < 1 || W < 1 || k_anchor < 1 || (n_rep > 0 && !row_ptr_b)) return CALIBATT_ERR_ARG;
+  const int64_t units_b = static_cast<int64_t>(n_rep) * anchor_blocks(frames, W, k_anchor);
+  if (row_ptr_b && (row_ptr_b[0] < 0 || row_ptr_b[units_b] < row_ptr_b[0])) return CALIBATT_ERR_CSR;
+  return balance_plan(work_list, n_work, row_ptr, heads, nb, row_ptr_b, units_b, n_slots);
 }
 
 int calibatt_shard_heads(const int32_t* row_ptr_host, int heads, int nb, const int32_t* rep_heads_host, int n_rep,
@@ -356,11 +375,12 @@ int calibatt_shard_heads(const int32_t* row_ptr_host, int heads, int nb, const i
   return CALIBATT_OK;
 }
 
-int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v, int heads,
-                            int frames, int H, int W, int d, int k_anchor, float scale, const int32_t* row_ptr,
-                            const int32_t* col_idx, int64_t nnz, const int32_t* rep_heads, int32_t n_rep,
-                            const int32_t* work_list, int32_t n_work, calibatt_bf16* o, float* lse, void* ws,
-                            size_t ws_bytes, calibatt_stream_t stream) {
+namespace {
+int mixed_attn(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v, int heads, int frames, int H,
+               int W, int d, int k_anchor, float scale, const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
+               const int32_t* rep_heads, int32_t n_rep, const int32_t* row_ptr_b, const int32_t* col_idx_b,
+               int64_t nnz_b, const int32_t* work_list, int32_t n_work, calibatt_bf16* o, float* lse, void* ws,
+               size_t ws_bytes, calibatt_stream_t stream) {
   if (!v || !o || frames < 1 || H < 1 || W < 1) return CALIBATT_ERR_ARG;
   const int64_t n64 = static_cast<int64_t>(frames) * H * W;
   if (n64 > INT_MAX / 2) return CALIBATT_ERR_ARG;
@@ -400,7 +420,32 @@ int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, cons
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.n_out = n;
+  p.row_ptr_b = n_rep > 0 ? row_ptr_b : nullptr;
+  p.col_idx_b = n_rep > 0 ? col_idx_b : nullptr;
+  p.nnz_b = nnz_b;
   return launch_attention(0, q, n, heads, k, v, n, heads, p, st, n_rep > 0 ? ws : nullptr, p.n_q_b, n_rep);
+}
+}  // namespace
+
+int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v, int heads,
+                            int frames, int H, int W, int d, int k_anchor, float scale, const int32_t* row_ptr,
+                            const int32_t* col_idx, int64_t nnz, const int32_t* rep_heads, int32_t n_rep,
+                            const int32_t* work_list, int32_t n_work, calibatt_bf16* o, float* lse, void* ws,
+                            size_t ws_bytes, calibatt_stream_t stream) {
+  return mixed_attn(q, k, v, heads, frames, H, W, d, k_anchor, scale, row_ptr, col_idx, nnz, rep_heads, n_rep,
+                    nullptr, nullptr, 0, work_list, n_work, o, lse, ws, ws_bytes, stream);
+}
+
+int calibatt_mixed_masked_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v,
+                                   int heads, int frames, int H, int W, int d, int k_anchor, float scale,
+                                   const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
+                                   const int32_t* rep_heads, int32_t n_rep, const int32_t* row_ptr_b,
+                                   const int32_t* col_idx_b, int64_t nnz_b, const int32_t* work_list, int32_t n_work,
+                                   calibatt_bf16* o, float* lse, void* ws, size_t ws_bytes,
+                                   calibatt_stream_t stream) {
+  if (n_rep > 0 && (!row_ptr_b || nnz_b < 0 || (nnz_b > 0 && !col_idx_b))) return CALIBATT_ERR_ARG;
+  return mixed_attn(q, k, v, heads, frames, H, W, d, k_anchor, scale, row_ptr, col_idx, nnz, rep_heads, n_rep,
+                    row_ptr_b, col_idx_b, nnz_b, work_list, n_work, o, lse, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ host buffers
@@ -808,6 +853,99 @@ int calibatt_aggregate_masks(const uint16_t* counts, int n_inputs, int heads, in
   calibatt_rho_threshold(n_inputs, rho, &thr);
   return launch_aggregate(counts, static_cast<int64_t>(heads) * nb, nb, thr, mask, row_ptr, col_idx, nnz_cap, nnz,
                           static_cast<int32_t*>(ws), status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t calibatt_anchor_energy_workspace_size(int heads, int n_rep, int frames, int H, int W, int k_anchor) {
+  if (heads < 1 || n_rep < 1 || n_rep > heads || frames < 1 || H < 1 || W < 1 || k_anchor < 1 || k_anchor > H)
+    return 0;
+  const int64_t n = static_cast<int64_t>(frames) * H * W;
+  const int64_t nb = (n + 127) / 128;
+  const int64_t units = n_rep * anchor_blocks(frames, W, k_anchor);
+  if (n > INT_MAX / 2 || units > INT_MAX / 2 || nb > CALIBATT_MAX_CALIB_NB) return 0;
+  const size_t packed = calibatt_repeat_workspace_size(n_rep, frames, H, W, k_anchor);
+  const size_t energy = static_cast<size_t>(2 * score_grid(static_cast<int>(units))) * nb * 128 * sizeof(float2);
+  return packed + ((energy + 255) & ~static_cast<size_t>(255));
+}
+
+int calibatt_anchor_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int frames, int H, int W,
+                                 int d, int k_anchor, float scale, const int32_t* rep_heads, int32_t n_rep, void* ws,
+                                 size_t ws_bytes, float* energy, int fuse_select, double eps, uint8_t* mask,
+                                 int32_t* kept, uint16_t* counts, uint8_t* tie, double tie_window,
+                                 calibatt_stream_t stream) {
+  if (frames < 1 || H < 1 || W < 1 || !rep_heads || n_rep < 1 || n_rep > heads) return CALIBATT_ERR_ARG;
+  const int64_t n64 = static_cast<int64_t>(frames) * H * W;
+  if (n64 > INT_MAX / 2) return CALIBATT_ERR_ARG;
+  const int n = static_cast<int>(n64);
+  int rc = check_qkv(q, k, nullptr, nullptr, heads, n, d);
+  if (rc != CALIBATT_OK) return rc;
+  if (k_anchor < 1 || k_anchor > H) return CALIBATT_ERR_ARG;
+  if (k_anchor > kMaxAnchors) return CALIBATT_ERR_UNSUPPORTED;
+  const int nb = (n + 127) / 128;
+  if (nb > CALIBATT_MAX_CALIB_NB) return CALIBATT_ERR_UNSUPPORTED;
+  if (!scale_ok(scale) || !ws || std::isnan(eps) || std::isnan(tie_window)) return CALIBATT_ERR_ARG;
+  if (ws_bytes < calibatt_anchor_energy_workspace_size(heads, n_rep, frames, H, W, k_anchor)) return CALIBATT_ERR_ARG;
+  if (fuse_select && !mask && !kept && !counts && !tie) return CALIBATT_ERR_ARG;
+  if (!aligned16(ws) || (energy && !aligned4(energy)) || (kept && !aligned4(kept)) ||
+      (counts && (reinterpret_cast<uintptr_t>(counts) & 1u)))
+    return CALIBATT_ERR_ALIGN;
+  KernelParams p = base_params();
+  if (!p.status) return CALIBATT_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the anchor queries of the repeated heads, packed frame by frame
+  AnchorTable tab;
+  int32_t anchors[kMaxAnchors];
+  calibatt_anchor_rows(H, k_anchor, anchors);
+  for (int j = 0; j < k_anchor; ++j) tab.anchor[j] = anchors[j];
+  const int n_q_b = frames * k_anchor * W;
+  rc = launch_gather(q, n, heads, rep_heads, n_rep, H, W, k_anchor, tab, ws, p.status, st);
+  if (rc != CALIBATT_OK) return rc;
+  // their block energies over every key block, in one pass
+  const size_t packed = calibatt_repeat_workspace_size(n_rep, frames, H, W, k_anchor);
+  p.n_q = n_q_b;
+  p.nbq = (n_q_b + 127) / 128;
+  p.n_k = n;
+  p.nbk = nb;
+  p.heads_q = n_rep;
+  p.heads_kv = heads;
+  p.head_map = rep_heads;
+  p.n_units = n_rep * p.nbq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_out = n;
+  p.energy_ws = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + packed);
+  p.energy = energy;
+  p.fuse_select = fuse_select ? 1 : 0;
+  p.eps_fx = eps_to_fixed(eps);
+  p.mask = fuse_select ? mask : nullptr;
+  p.kept = fuse_select ? kept : nullptr;
+  p.counts = fuse_select ? counts : nullptr;
+  p.tie = fuse_select ? tie : nullptr;
+  p.tie_fx = tie_window_fixed(tie_window);
+  return launch_attention(3, ws, n_q_b, n_rep, k, nullptr, n, heads, p, st);
+}
+
+size_t calibatt_aggregate_rows_workspace_size(int64_t rows) {
+  if (rows < 1 || rows > INT_MAX / 2) return 0;
+  const size_t bytes = static_cast<size_t>(aggregate_scratch_ints(rows)) * sizeof(int32_t);
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+int calibatt_aggregate_mask_rows(const uint16_t* counts, int n_inputs, int64_t rows, int cols, double rho,
+                                 uint8_t* mask, int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap, int64_t* nnz,
+                                 void* ws, size_t ws_bytes, calibatt_stream_t stream) {
+  if (!counts || !mask || !row_ptr || !nnz || rows < 1 || cols < 1 || n_inputs < 1 || nnz_cap < 0 ||
+      (nnz_cap > 0 && !col_idx) || !std::isfinite(rho))
+    return CALIBATT_ERR_ARG;
+  if (rows > INT_MAX / 2 || rows * cols > INT_MAX) return CALIBATT_ERR_ARG;
+  if (!ws || ws_bytes < calibatt_aggregate_rows_workspace_size(rows)) return CALIBATT_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(counts) & 1u) || !aligned4(row_ptr) || (col_idx && !aligned4(col_idx)) ||
+      (reinterpret_cast<uintptr_t>(nnz) & 7u) || !aligned4(ws))
+    return CALIBATT_ERR_ALIGN;
+  int* status = status_word();
+  if (!status) return CALIBATT_ERR_CUDA;
+  int32_t thr = 0;
+  calibatt_rho_threshold(n_inputs, rho, &thr);
+  return launch_aggregate(counts, rows, cols, thr, mask, row_ptr, col_idx, nnz_cap, nnz, static_cast<int32_t*>(ws),
+                          status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -71,6 +71,29 @@ struct AttnLayout {
   static constexpr int kDynSmem = kBytes + 1024;  // + alignment slack
 };
 
+// Output rows of a query row of a unit: the row itself (block-sparse unit),
+// or the band of rows its anchor row is broadcast to (anchor-query unit of a
+// repeated head: same frame, same column); none for a padded row.
+__device__ __forceinline__ void unit_dst(const KernelParams& p, const Unit& u, int qrow, bool row_valid,
+                                         int64_t& dst0, int& n_dst, int& dst_stride) {
+  dst0 = 0;
+  n_dst = 0;
+  dst_stride = 0;
+  if (!row_valid) return;
+  if (u.rep) {
+    const int kw = p.rep_k * p.rep_W;
+    const int f = qrow / kw, rem = qrow % kw;
+    const int ja = rem / p.rep_W, c = rem % p.rep_W;
+    const int lo = p.band_lo[ja], hi = p.band_hi[ja];
+    dst0 = static_cast<int64_t>(f) * p.rep_H * p.rep_W + static_cast<int64_t>(lo) * p.rep_W + c;
+    n_dst = hi - lo;
+    dst_stride = p.rep_W;
+  } else {
+    dst0 = qrow;
+    n_dst = 1;
+  }
+}
+
 template <bool SW>  // SW: the polling wait form of short (test) wait limits
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qb,
@@ -269,14 +292,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int qrow = u.r * 128 + row;
       const bool row_valid = qrow < (u.rep ? p.n_q_b : p.n_q);
       if (u.nnz == 0) {
-        // no kept block: O = 0, lse = -inf
-        if (row_valid) {
-          uint32_t z[16];
+        // no kept block: O = 0, lse = -inf (for every row a repeated head's
+        // anchor row feeds)
+        int64_t dst0;
+        int n_dst, dst_stride;
+        unit_dst(p, u, qrow, row_valid, dst0, n_dst, dst_stride);
+        __nv_bfloat16* obase = p.o + static_cast<int64_t>(u.hkv) * p.n_out * 128;
+        uint32_t z[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) z[i] = 0;
-          for (int c = 0; c < 4; ++c)
-            store_row_chunk(p.o + (static_cast<int64_t>(u.hkv) * p.n_out + qrow) * 128 + c * 32, z);
-          if (p.lse) p.lse[static_cast<int64_t>(u.hkv) * p.n_out + qrow] = -INFINITY;
+        for (int i = 0; i < 16; ++i) z[i] = 0;
+        for (int q = 0; q < n_dst; ++q) {
+          const int64_t d = dst0 + static_cast<int64_t>(q) * dst_stride;
+          for (int c = 0; c < 4; ++c) store_row_chunk(obase + d * 128 + c * 32, z);
+          if (p.lse) p.lse[static_cast<int64_t>(u.hkv) * p.n_out + d] = -INFINITY;
         }
         continue;
       }
@@ -343,23 +371,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const float lse_val = (m_run + log2f(l_run)) * kLn2;
-      // destination rows: one per query (sparse), or a band of rows (repeat)
-      int64_t dst0 = 0;
-      int n_dst = 0, dst_stride = 0;
-      if (row_valid) {
-        if (u.rep) {
-          const int kw = p.rep_k * p.rep_W;
-          const int f = qrow / kw, rem = qrow % kw;
-          const int ja = rem / p.rep_W, c = rem % p.rep_W;
-          const int lo = p.band_lo[ja], hi = p.band_hi[ja];
-          dst0 = static_cast<int64_t>(f) * p.rep_H * p.rep_W + static_cast<int64_t>(lo) * p.rep_W + c;
-          n_dst = hi - lo;
-          dst_stride = p.rep_W;
-        } else {
-          dst0 = qrow;
-          n_dst = 1;
-        }
-      }
+      int64_t dst0;
+      int n_dst, dst_stride;
+      unit_dst(p, u, qrow, row_valid, dst0, n_dst, dst_stride);
       __nv_bfloat16* obase = p.o + static_cast<int64_t>(u.hkv) * p.n_out * 128;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {

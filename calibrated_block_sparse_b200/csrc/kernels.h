@@ -32,6 +32,11 @@ struct KernelParams {
   // every key block, and head_map_b gives their K/V/O head. nbq_b = 0: none.
   int n_q_b, nbq_b, heads_q_b;
   const int32_t* head_map_b;
+  // optional skip list of the anchor-query units ([heads_q_b * nbq_b + 1]
+  // global offsets into col_idx_b, columns ascending); NULL: every key block
+  const int32_t* row_ptr_b;
+  const int32_t* col_idx_b;
+  int64_t nnz_b;
   // repeated heads: a packed anchor query q = f*(k*W) + j*W + c writes rows
   // band_lo[j] .. band_hi[j]-1 of frame f, column c
   int rep_H, rep_W, rep_k;

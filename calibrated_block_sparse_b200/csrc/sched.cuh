@@ -44,7 +44,8 @@ __device__ __forceinline__ bool load_unit(const KernelParams& p, int idx, Unit& 
   u.write = true;
   u.rep = false;
   if (code >= n_a && p.nbq_b > 0 && code - n_a < p.heads_q_b * p.nbq_b) {
-    // anchor-query unit: every key block, K/V/O head from head_map_b
+    // anchor-query unit: K/V/O head from head_map_b; every key block, or the
+    // blocks of its own skip list
     const int c = code - n_a;
     u.rep = true;
     u.hq = c / p.nbq_b;
@@ -57,6 +58,16 @@ __device__ __forceinline__ bool load_unit(const KernelParams& p, int idx, Unit& 
     }
     u.base = 0;
     u.nnz = u.write ? p.nbk : 0;
+    if (u.write && p.row_ptr_b) {
+      const int a = __ldg(p.row_ptr_b + c), b = __ldg(p.row_ptr_b + c + 1);
+      if (a < 0 || b < a || static_cast<int64_t>(b) > p.nnz_b) {
+        record_error(p.status, CALIBATT_ERR_CSR);
+        u.nnz = 0;
+      } else {
+        u.base = a;
+        u.nnz = b - a;
+      }
+    }
     return true;
   }
   if (code < 0 || code >= n_a) {
@@ -95,8 +106,9 @@ __device__ __forceinline__ bool load_unit(const KernelParams& p, int idx, Unit& 
 
 // Key block of the j-th kept tile; out-of-range entries are clamped and reported.
 __device__ __forceinline__ int block_col(const KernelParams& p, const Unit& u, int j) {
-  if (!p.col_idx || u.rep) return j;
-  int c = __ldg(p.col_idx + u.base + j);
+  const int32_t* ci = u.rep ? p.col_idx_b : p.col_idx;
+  if (!ci) return j;
+  int c = __ldg(ci + u.base + j);
   if (c < 0 || c >= p.nbk) {
     record_error(p.status, CALIBATT_ERR_CSR);
     c = c < 0 ? 0 : p.nbk - 1;

@@ -176,6 +176,14 @@ int calibatt_repeat_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, con
 int calibatt_balance_plan(int32_t* work_list, int32_t n_work, const int32_t* row_ptr, int heads, int nb,
                           int n_slots);
 
+/* calibatt_balance_plan for a work list of calibatt_mixed_masked_attn_fwd:
+ * the cost of an anchor-query unit is its kept blocks in the anchor skip list
+ * row_ptr_b (host int32 [n_rep * ceil(frames*k_anchor*W / 128) + 1]) instead
+ * of every key block; row_ptr_b may be NULL when n_rep = 0. Same layout rule
+ * and result guarantees as calibatt_balance_plan. */
+int calibatt_balance_mixed_plan(int32_t* work_list, int32_t n_work, const int32_t* row_ptr, int heads, int nb,
+                                const int32_t* row_ptr_b, int n_rep, int frames, int W, int k_anchor, int n_slots);
+
 /* Work list for calibatt_mixed_attn_fwd: first the anchor-query units of the
  * repeated heads, ceil(frames*k_anchor*W / 128) per head rep_heads[i] (codes
  * heads*nb + i*ceil(..) + b, each taking every key block), then head by head
@@ -203,6 +211,32 @@ int calibatt_mixed_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, cons
                             const int32_t* col_idx, int64_t nnz, const int32_t* rep_heads, int32_t n_rep,
                             const int32_t* work_list, int32_t n_work, calibatt_bf16* o, float* lse, void* ws,
                             size_t ws_bytes, calibatt_stream_t stream);
+
+/* calibatt_mixed_attn_fwd with a block mask on the repeated heads' anchor
+ * rows (explainer §三 makes both run-time decisions per (t, l, h): a head's
+ * skip list and its spatial repetition; the pages do not combine them, and
+ * this call applies both): the anchor queries of repeated head rep_heads[i],
+ * taken frame by frame (packed row f*k*W + j*W + c is token
+ * f*H*W + a_j*W + c) and grouped into blocks of 128, attend only to the key
+ * blocks of their block's row in the anchor skip list; every row still takes
+ * its nearest anchor row's output. An anchor block with no kept block gives
+ * O = 0 and lse = -inf to every row it feeds.
+ *   row_ptr_b : device int32 [n_rep * ceil(frames*k_anchor*W / 128) + 1],
+ *               global offsets into col_idx_b (rows of repeated head i start
+ *               at i * ceil(frames*k_anchor*W / 128))
+ *   col_idx_b : device int32 [nnz_b], ascending within a row, in [0, nb)
+ * Calibrate it with calibatt_anchor_block_energy and
+ * calibatt_aggregate_mask_rows. Other arguments as in
+ * calibatt_mixed_attn_fwd (work list from calibatt_build_mixed_plan, laid out
+ * by calibatt_balance_mixed_plan); a malformed anchor list is clamped and
+ * reported as CALIBATT_ERR_CSR through calibatt_get_status. */
+int calibatt_mixed_masked_attn_fwd(const calibatt_bf16* q, const calibatt_bf16* k, const calibatt_bf16* v,
+                                   int heads, int frames, int H, int W, int d, int k_anchor, float scale,
+                                   const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
+                                   const int32_t* rep_heads, int32_t n_rep, const int32_t* row_ptr_b,
+                                   const int32_t* col_idx_b, int64_t nnz_b, const int32_t* work_list, int32_t n_work,
+                                   calibatt_bf16* o, float* lse, void* ws, size_t ws_bytes,
+                                   calibatt_stream_t stream);
 
 /* Head sharding of one attention call over n_ranks GPUs (host). A head's
  * output depends only on its own q, k, v, so ranks need no exchange; the
@@ -299,6 +333,30 @@ int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, 
                                 uint8_t* mask, int32_t* kept, uint16_t* counts, uint8_t* tie, double tie_window,
                                 float* pix_energy, int pix_W, calibatt_stream_t stream);
 
+/* Device workspace bytes of calibatt_anchor_block_energy (0 on bad sizes). */
+size_t calibatt_anchor_energy_workspace_size(int heads, int n_rep, int frames, int H, int W, int k_anchor);
+
+/* Block energies of the repeated heads' anchor queries (the calibration of
+ * the anchor-row masks of calibatt_mixed_masked_attn_fwd; explainer §三 step
+ * 2, taken over anchor queries): the anchor queries of head rep_heads[i],
+ * packed frame by frame as in calibatt_mixed_masked_attn_fwd and grouped into
+ * nbq = ceil(frames*k_anchor*W / 128) blocks, against every key block of the
+ * head, in one pass over the keys:
+ *   E[i][r][c] = (1 / |I_r|) * sum_{a in packed block r, j in block c} P_aj,
+ * P = softmax(scale * Q K^T) over all n keys. With fuse_select, the greedy
+ * selection of calibatt_select_mask at eps runs on every finished row.
+ *   rep_heads : device int32 [n_rep], in [0, heads)
+ *   ws        : device scratch of calibatt_anchor_energy_workspace_size bytes,
+ *               16-byte aligned (the packed queries, then the pass's sums)
+ *   energy    : device fp32 [n_rep][nbq][nb] or NULL
+ *   mask, kept, counts, tie : as in calibatt_block_energy, with n_rep*nbq rows
+ * Requires nb <= CALIBATT_MAX_CALIB_NB. */
+int calibatt_anchor_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int heads, int frames, int H, int W,
+                                 int d, int k_anchor, float scale, const int32_t* rep_heads, int32_t n_rep, void* ws,
+                                 size_t ws_bytes, float* energy, int fuse_select, double eps, uint8_t* mask,
+                                 int32_t* kept, uint16_t* counts, uint8_t* tie, double tie_window,
+                                 calibatt_stream_t stream);
+
 /* Greedy eps selection (explainer §三, step 3) on rows of block energies:
  * order the row's blocks by energy descending (equal energies: lower column
  * first) and keep the shortest prefix whose running sum reaches eps. The sum
@@ -343,6 +401,18 @@ size_t calibatt_aggregate_workspace_size(int heads, int nb);
 int calibatt_aggregate_masks(const uint16_t* counts, int n_inputs, int heads, int nb, double rho, uint8_t* mask,
                              int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, void* ws,
                              size_t ws_bytes, calibatt_stream_t stream);
+
+/* Workspace bytes needed by calibatt_aggregate_mask_rows for `rows` rows. */
+size_t calibatt_aggregate_rows_workspace_size(int64_t rows);
+
+/* calibatt_aggregate_masks for any number of mask rows of `cols` columns
+ * (for example the n_rep * nbq anchor rows of calibatt_anchor_block_energy):
+ * keep cell (r, c) where counts[r][c] / n_inputs >= rho, and build the CSR
+ * skip list of the rows (row_ptr [rows + 1], global offsets, columns
+ * ascending). Outputs, capacity and errors as in calibatt_aggregate_masks. */
+int calibatt_aggregate_mask_rows(const uint16_t* counts, int n_inputs, int64_t rows, int cols, double rho,
+                                 uint8_t* mask, int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap, int64_t* nnz,
+                                 void* ws, size_t ws_bytes, calibatt_stream_t stream);
 
 /* ---------------------------------------------------------------- spatial repetition */
 

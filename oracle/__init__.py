@@ -67,6 +67,8 @@ def _load():
             lib.oracle_binarize_counts.restype = None
             lib.oracle_mask_to_csr.argtypes = [P, i32, i64, P, P]
             lib.oracle_mask_to_csr.restype = i64
+            lib.oracle_mask_rows_to_csr.argtypes = [P, i64, i64, P, P]
+            lib.oracle_mask_rows_to_csr.restype = i64
             lib.oracle_eps_schedule.argtypes = [f64, f64, f64, f64, f64]
             lib.oracle_eps_schedule.restype = f64
             lib.oracle_pixel_row_energy.argtypes = [P, P, i32, i32, i32, i32, i32, i32, f64, P, i64, P, i32]
@@ -241,6 +243,19 @@ def mask_to_csr(mask):
     row_ptr = np.empty(h * nb + 1, np.int32)
     col_idx = np.empty(int(mask.sum()), np.int32)
     nnz = _load().oracle_mask_to_csr(_ptr(mask), h, nb, _ptr(row_ptr), _ptr(col_idx))
+    assert nnz == col_idx.size
+    return row_ptr, col_idx
+
+
+def mask_rows_to_csr(mask):
+    """Skip list of the rows of a mask [..., cols] (any number of rows): per
+    row the kept columns, ascending, as CSR with global offsets."""
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    cols = mask.shape[-1]
+    rows = mask.size // cols
+    row_ptr = np.empty(rows + 1, np.int32)
+    col_idx = np.empty(int(mask.sum()), np.int32)
+    nnz = _load().oracle_mask_rows_to_csr(_ptr(mask), rows, cols, _ptr(row_ptr), _ptr(col_idx))
     assert nnz == col_idx.size
     return row_ptr, col_idx
 

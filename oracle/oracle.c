@@ -379,6 +379,20 @@ int64_t oracle_mask_to_csr(const uint8_t *mask, int heads, int64_t nb, int32_t *
     return nnz;
 }
 
+/* The same skip list for any number of mask rows of `cols` columns (for
+ * example the anchor-block rows of repeated heads). */
+int64_t oracle_mask_rows_to_csr(const uint8_t *mask, int64_t rows, int64_t cols, int32_t *row_ptr,
+                                int32_t *col_idx) {
+    int64_t nnz = 0;
+    for (int64_t row = 0; row < rows; ++row) {
+        row_ptr[row] = (int32_t)nnz;
+        for (int64_t c = 0; c < cols; ++c)
+            if (mask[row * cols + c]) col_idx[nnz++] = (int32_t)c;
+    }
+    row_ptr[rows] = (int32_t)nnz;
+    return nnz;
+}
+
 /* ------------------------------------------------------------------------ */
 /* 6. Energy threshold schedule (explainer §三): eps(t) = A + (C - A) e^{-kt/T} */
 /*    high (C) at the early, high-noise steps, relaxing towards A.           */

@@ -217,6 +217,18 @@ def test_bank_index_on_the_host(binding):
                                             4, None, 0, 8, fake, fake, fake, fake, None, fake, 4, None) == -1
     assert lib.calibatt_mixed_attn_fwd_host(None, fake, fake, fake, None, 2, 2, 8, 16, 128, 5, 0.1, fake, fake, fake,
                                             4, None, 0, 8, fake, fake, fake, fake, None, fake, 1 << 30, None) == -1
+    # anchor-row masks: missing anchor skip list, bad sizes, short workspace
+    assert lib.calibatt_mixed_masked_attn_fwd(fake, fake, fake, 2, 2, 8, 16, 128, 5, 0.1, fake, fake, 4, fake, 1,
+                                              None, None, 0, fake, 2, fake, None, fake, 1 << 30, None) == -1
+    assert lib.calibatt_anchor_energy_workspace_size(2, 3, 2, 8, 16, 5) == 0      # more repeated heads than heads
+    assert lib.calibatt_anchor_energy_workspace_size(2, 1, 2, 8, 16, 9) == 0      # k above H
+    assert lib.calibatt_anchor_block_energy(fake, fake, 2, 2, 8, 16, 128, 5, 0.1, fake, 1, fake, 16, None, 1, 0.9,
+                                            fake, None, None, None, 0.0, None) == -1
+    assert lib.calibatt_anchor_block_energy(fake, fake, 2, 2, 8, 16, 128, 5, 0.1, None, 1, fake, 1 << 30, None, 0,
+                                            0.9, None, None, None, None, 0.0, None) == -1
+    assert lib.calibatt_aggregate_rows_workspace_size(0) == 0
+    assert lib.calibatt_aggregate_mask_rows(fake, 4, 10, 16, 0.5, fake, fake, fake, 160, fake, fake, 4, None) == -1
+    assert lib.calibatt_aggregate_mask_rows(fake, 4, 0, 16, 0.5, fake, fake, fake, 160, fake, fake, 4096, None) == -1
     # keep-rate histogram arguments
     assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 0, P(0x100000), None) == -1
     assert lib.calibatt_keep_histogram(P(0x100000), 1, 16, 8, P(0x100004), None) == -3
@@ -322,3 +334,18 @@ def test_balance_plan_edge_cases(binding):
     lib = binding.load()
     assert lib.calibatt_balance_plan(binding._ptr(w), 3, binding._ptr(rp), 1, 3, 1) == -1  # fewer than 2 slots
     assert lib.calibatt_balance_plan(None, 3, binding._ptr(rp), 1, 3, 8) == -1
+
+
+def test_balance_mixed_plan_costs_anchor_units_by_their_skip_list(binding):
+    """Anchor units with few kept blocks weigh less: the balanced list is a
+    permutation within rounds, and with two slots the heavy anchor unit and
+    the light ones are spread so that both slots carry similar work."""
+    heads, nb, F, W, kk = 2, 4, 1, 256, 1   # one repeated head: 2 anchor blocks
+    rp = np.array([0, 4, 8, 12, 16, 20, 24, 28, 32], np.int32)  # every block kept
+    rpb = np.array([0, 4, 5], np.int32)   # anchor block 0 keeps 4 blocks, block 1 keeps 1
+    work = binding.build_mixed_plan(rp, heads, nb, [1], F, 4, W, kk)
+    assert sorted(work.tolist()) == sorted(list(range(0, 4)) + [heads * nb, heads * nb + 1])
+    bal = binding.balance_mixed_plan(work, rp, heads, nb, rpb, 1, F, W, kk, n_slots=2)
+    assert sorted(bal.tolist()) == sorted(work.tolist())
+    with pytest.raises(binding.CalibattError):
+        binding.balance_mixed_plan(work, rp, heads, nb, None, 1, F, W, kk, n_slots=2)

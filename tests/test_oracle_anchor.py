@@ -126,3 +126,16 @@ def test_k_outside_range_is_refused(oracle):
     q, k, v = _rand(1, 2 * 3 * 8, seed=9)
     with pytest.raises(ValueError):
         oracle.anchor_block_energy(q, k, 2, 3, 8, k_anchor=4)
+
+
+def test_row_skip_list_equals_the_square_one(oracle):
+    mask = synth.random_mask(3, 11, 0.4, seed=10)
+    rp, ci = oracle.mask_rows_to_csr(mask)
+    rp2, ci2 = oracle.mask_to_csr(mask)
+    np.testing.assert_array_equal(rp, rp2)
+    np.testing.assert_array_equal(ci, ci2)
+    rect = mask[:, :7, :].copy()  # 7 rows of 11 columns per head
+    rp3, ci3 = oracle.mask_rows_to_csr(rect)
+    assert rp3.size == 3 * 7 + 1 and rp3[-1] == rect.sum()
+    for r in range(21):
+        np.testing.assert_array_equal(ci3[rp3[r]:rp3[r + 1]], np.nonzero(rect.reshape(21, 11)[r])[0])
