@@ -413,6 +413,63 @@ class Step:
         return out
 
 
+def anchor_masked_step(binding, step, dev, stream, pk, reps, n_in, eps):
+    """The step with block masks on the repeated heads' anchor rows: the anchor
+    queries calibrated over n_in seeded inputs at eps (single-pass energy with
+    fused selection), aggregated at rho = 0.5, then the masked mixed launch on
+    the step's inputs. Kept-tile flops count each kept anchor tile by its valid
+    anchor rows and key columns."""
+    wl = step.wl
+    rep = step.rep
+    if not rep:
+        return None
+    heads, nb, n = wl.heads, wl.nb, wl.n
+    nbq = binding.anchor_blocks(wl.F, wl.W, wl.k_anchor)
+    rep_t = step.rep_t
+    counts = torch.zeros((len(rep), nbq, nb), dtype=torch.uint16, device=dev)
+    ws = torch.empty(binding.load().calibatt_anchor_energy_workspace_size(heads, len(rep), wl.F, wl.H, wl.W,
+                                                                          wl.k_anchor), dtype=torch.uint8, device=dev)
+    ms_cal = 0.0
+    for p in range(n_in):
+        q, k, _ = synth.qkv(wl, p, with_v=False, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        binding.anchor_block_energy(q, k, wl.F, wl.H, wl.W, rep_t, k_anchor=wl.k_anchor, eps=eps, energy=False,
+                                    counts=counts, ws=ws, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        ms_cal += e0.elapsed_time(e1)
+        del q, k
+    del ws
+    mask_b, rpb, cib, _ = binding.aggregate_mask_rows(counts, n_in, 0.5, stream=stream)
+    mb = mask_b.cpu().numpy()
+    rpb_h = rpb.cpu().numpy()
+    work = binding.build_mixed_plan(step.row_ptr_h, heads, nb, rep, wl.F, wl.H, wl.W, wl.k_anchor)
+    work = torch.from_numpy(binding.balance_mixed_plan(work, step.row_ptr_h, heads, nb, rpb_h, len(rep), wl.F, wl.W,
+                                                       wl.k_anchor)).to(dev)
+
+    def call():
+        binding.mixed_masked_attn_fwd(step.q, step.k, step.v, wl.F, wl.H, wl.W, step.row_ptr, step.col_idx, rep_t,
+                                      rpb, cib, work, wl.k_anchor, o=step.o, lse=step.lse, ws=step.ws, stream=stream)
+
+    for _ in range(3):
+        call()
+    ms = cuda_time(call, reps, stream)
+    binding.check_status(what="anchor-masked step")
+    step()  # restore the unmasked call's output in the shared buffers
+    vq = valid_sizes(wl.F * wl.k_anchor * wl.W, nbq)
+    vk = valid_sizes(n, nb)
+    f_anchor = float(4 * D * sum(int((mb[i].astype(np.int64) * np.outer(vq, vk)).sum()) for i in range(len(rep))))
+    flops = step.f_sparse + f_anchor
+    tflops = flops / (ms * 1e-3) / 1e12
+    f_alg = 2.0 * D * (wl.F * wl.k_anchor * wl.W) * n * len(rep)
+    return {"calibration": {"inputs": n_in, "eps": eps, "rho": 0.5, "kernel": "calibatt_anchor_block_energy",
+                            "ms_per_input": ms_cal / n_in, "energy_tflops": f_alg / (ms_cal / n_in * 1e-3) / 1e12},
+            "anchor_block_sparsity": 1.0 - float(mb.mean()), "ms_per_call": ms, "kept_tile_tflops": tflops,
+            "frac_of_bf16_burst": frac_of(tflops, pk, "bf16_tflops"), "kept_tile_flops": flops,
+            "speedup_vs_unmasked_step": None}
+
+
 def attention_config(binding, name, dev, pk, reps, with_library):
     """Skip lists (calibrated or random), then one attention call timed, and
     the same kernel at 0 % sparsity, on a stream of its own (CUDA graphs time
@@ -448,6 +505,11 @@ def _attention_config(binding, name, dev, stream, pk, reps, with_library):
     step()  # the dense run wrote the same output buffers: restore the call's result
     out = step.summary(ms, dense_ms, pk, lib)
     out["skip_lists"] = calib
+    if step.rep:
+        n_cal, eps_cal = synth.CALIBRATION[name]
+        am = anchor_masked_step(binding, step, dev, stream, pk, reps, n_cal, eps_cal)
+        am["speedup_vs_unmasked_step"] = ms / am["ms_per_call"]
+        out["anchor_masked"] = am
     return out, step
 
 
@@ -833,6 +895,11 @@ def run_ours(args, world, rank, local):
     # of a one-GPU run; each is timed on its own after the timed region)
     configs = {args.workload: step.summary(ms_step, dense_ms, pk, lib_dense)}
     configs[args.workload]["skip_lists"] = calib_info
+    if world == 1 and not args.heads and step.rep and args.workload == "wan720":
+        # anchor-row masks of the repeated heads, calibrated at eps(T/2)
+        am = anchor_masked_step(binding, step, dev, stream, pk, reps, 4, synth.CALIBRATION["wan480"][1])
+        am["speedup_vs_unmasked_step"] = ms_step / am["ms_per_call"]
+        configs[args.workload]["anchor_masked"] = am
     calib = sweep = fp8 = tiny_step = None
     if world == 1 and not args.heads:
         for name in (args.configs or []):
