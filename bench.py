@@ -731,6 +731,23 @@ def fp8_probe(binding, name, n_in, dev, stream):
             "aggregated_cells": heads * nb * nb}
 
 
+def run_calib_only(args):
+    """Only the calibration kernels (energy, selection, aggregation, profiles,
+    spatial score) on the first --heads heads of the Wan-720p shape: the small
+    case that ncu captures of those kernels run."""
+    from calibrated_block_sparse_b200 import binding
+    binding.load()
+    import dataclasses
+    wl = synth.WORKLOADS["calib720"]
+    wl = dataclasses.replace(wl, heads=args.heads or wl.heads)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    pk, _ = peaks()
+    q, k, _ = synth.qkv(wl, 0, with_v=False, device=dev)
+    out = calibration_kernels(binding, wl, q, k, dev, stream, pk)
+    print(json.dumps({"calibration_kernels": out}), flush=True)
+
+
 def run_ours(args, world, rank, local):
     from calibrated_block_sparse_b200 import binding
     binding.load()
@@ -1004,6 +1021,8 @@ def main():
                     help="other workloads reported under 'configs' (comma-separated; 'none' for none)")
     ap.add_argument("--sweep-inputs", type=int, default=64, help="calibration inputs of the sweep workload")
     ap.add_argument("--no-fp8-probe", dest="fp8_probe", action="store_false")
+    ap.add_argument("--calib-only", action="store_true",
+                    help="only the calibration kernels on --heads heads of the Wan-720p shape (profiling case)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="dram bytes per launch of the sparse kernel from an ncu capture")
     args = ap.parse_args()
@@ -1013,6 +1032,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.calib_only:
+            run_calib_only(args)
         else:
             run_ours(args, world, rank, local)
     finally:
