@@ -268,10 +268,11 @@ def graph_time(fn, reps, stream):
 
 
 # DRAM bytes per kept tile of the attention kernel: one ncu capture of the
-# 5-head Wan-720p launch (heads 0-3 block-sparse, head 4 repeated), 565.2 MB
-# of dram__bytes_read.sum + dram__bytes_write.sum over its 514 058 kept tiles;
-# the roofline's traffic scales it by the tiles of the timed launch.
-TRAFFIC_PER_TILE = 565.24e6 / 514058
+# 5-head Wan-720p launch (heads 0-3 block-sparse, head 4 repeated), 538.9 MB
+# read + 89.5 MB written (dram__bytes_read.sum + dram__bytes_write.sum) over
+# its 514 058 kept tiles; the roofline's traffic scales it by the tiles of
+# the timed launch.
+TRAFFIC_PER_TILE = 628.43e6 / 514058
 
 
 def frac_of(achieved, pk, key):
