@@ -43,90 +43,196 @@ __global__ void accumulate_kernel(const uint8_t* __restrict__ mask, int64_t cell
 }
 
 // ------------------------------------------------------------------ aggregation
-// Two launches over CTAs of kAggRows block-rows (one warp per row):
-//  1. binarize: counts >= threshold -> mask row, the row's kept count, and
-//     the CTA's total;
-//  2. compact: each CTA adds up the totals of the CTAs before it (all final
-//     once the first launch is done: no cross-CTA waiting), scans its own
-//     rows' counts into row_ptr (global offsets), and writes each row's kept
-//     columns in ascending order. The last CTA writes the grand total.
-// Scratch: row_cnt[rows] then cta_sum[ceil(rows / kAggRows)].
-constexpr int kAggRows = 32;  // = warps per CTA = lanes of a warp (partials are read one per lane)
+// The CSR skip list of a mask holds its kept cells in flat (row-major) order:
+// cell (row, col) goes to col_idx at its rank among the kept cells, and
+// row_ptr[row] is the rank of cell (row, 0). Two launches over CTAs that each
+// own one contiguous span of the flat arrays:
+//  1. binarize: counts >= threshold -> mask, and the span's kept total;
+//  2. compact: the totals of the spans before it (all final once the first
+//     launch is done: no cross-CTA waiting) give the span's first rank; the
+//     span is then walked in rounds of kAggRound cells, lane chunks of
+//     kAggChunk cells ranked by a block scan per round; each warp stages its
+//     kept columns in shared memory and stores them as one coalesced run.
+//     The last CTA writes the grand total.
+// A span is a whole number of rounds, so with 16-byte aligned arrays every
+// lane chunk is one 16-byte mask vector and two 16-byte count vectors.
+// Scratch: one total per span.
+constexpr int kAggThreads = 256;
+constexpr int kAggWarps = kAggThreads / 32;
+constexpr int kAggChunk = 16;
+constexpr int kAggRound = kAggThreads * kAggChunk;
+constexpr int64_t kAggFill = 148 * 8;  // CTAs that fill the SMs at 8 per SM
 
-__global__ void __launch_bounds__(kAggRows * 32) binarize_kernel(const uint16_t* __restrict__ counts, int64_t rows,
-                                                                 int nb, int threshold, uint8_t* mask,
-                                                                 int32_t* row_cnt, int32_t* cta_sum) {
-  __shared__ int wsum[kAggRows];
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kAggRows + w;
-  int cnt = 0;
-  if (row < rows) {
-    const uint16_t* src = counts + row * nb;
-    uint8_t* dst = mask + row * nb;
-#pragma unroll 4
-    for (int c = lane; c < nb; c += 32) {
-      const uint8_t k = src[c] >= threshold ? 1 : 0;
-      dst[c] = k;
-      cnt += k;
-    }
-    cnt = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
-    if (lane == 0) row_cnt[row] = cnt;
+// 0/1 bytes for four counts (two per word) against the threshold pair t2.
+__device__ __forceinline__ uint32_t keep4(uint32_t a, uint32_t b, uint32_t t2, bool none) {
+  if (none) return 0u;
+  const uint32_t fa = __vcmpgeu2(a, t2) & 0x00010001u, fb = __vcmpgeu2(b, t2) & 0x00010001u;
+  return __byte_perm(fa, fb, 0x6420);
+}
+
+// One lane chunk's 0/1 mask bytes -> 16-bit kept bitmap (bit j = cell j).
+// Within a word, bytes b0..b3 times 0x01020408 land b_i on bit 24 + i, every
+// other partial product on a bit below 24 or past 31, with no carries.
+__device__ __forceinline__ uint32_t chunk_bits(const uint32_t (&m)[4]) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) bits |= (((m[q] & 0x01010101u) * 0x01020408u) >> 24) << (4 * q);
+  return bits;
+}
+
+template <bool kVec>
+__device__ __forceinline__ int binarize_chunk(const uint16_t* __restrict__ counts, uint8_t* __restrict__ mask,
+                                              int64_t g, int64_t s1, const uint4& a, const uint4& b, int threshold,
+                                              uint32_t t2, bool none) {
+  if (kVec && g + kAggChunk <= s1) {
+    uint4 m;
+    m.x = keep4(a.x, a.y, t2, none);
+    m.y = keep4(a.z, a.w, t2, none);
+    m.z = keep4(b.x, b.y, t2, none);
+    m.w = keep4(b.z, b.w, t2, none);
+    *reinterpret_cast<uint4*>(mask + g) = m;
+    return __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
   }
+  int cnt = 0;
+  for (int j = 0; j < kAggChunk && g + j < s1; ++j) {
+    const int k = counts[g + j] >= threshold ? 1 : 0;
+    mask[g + j] = static_cast<uint8_t>(k);
+    cnt += k;
+  }
+  return cnt;
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(kAggThreads) binarize_kernel(const uint16_t* __restrict__ counts, int64_t cells,
+                                                               int64_t span, int threshold,
+                                                               uint8_t* __restrict__ mask,
+                                                               int32_t* __restrict__ span_sum) {
+  __shared__ int wsum[kAggWarps];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t s0 = static_cast<int64_t>(blockIdx.x) * span;
+  const int64_t s1 = s0 + span < cells ? s0 + span : cells;
+  const bool none = threshold > 65535;  // counts are 16-bit
+  const uint32_t t2 = static_cast<uint32_t>(threshold > 0 ? threshold : 0) * 0x10001u;
+  int cnt = 0;
+  // two rounds per step, both rounds' loads in flight before either is used
+  for (int64_t g = s0 + threadIdx.x * kAggChunk; g < s1; g += 2 * kAggRound) {
+    const int64_t h = g + kAggRound;
+    uint4 a0 = {}, b0 = {}, a1 = {}, b1 = {};
+    if (kVec && g + kAggChunk <= s1) {
+      a0 = *reinterpret_cast<const uint4*>(counts + g);
+      b0 = *reinterpret_cast<const uint4*>(counts + g + 8);
+    }
+    if (kVec && h + kAggChunk <= s1) {
+      a1 = *reinterpret_cast<const uint4*>(counts + h);
+      b1 = *reinterpret_cast<const uint4*>(counts + h + 8);
+    }
+    cnt += binarize_chunk<kVec>(counts, mask, g, s1, a0, b0, threshold, t2, none);
+    if (h < s1) cnt += binarize_chunk<kVec>(counts, mask, h, s1, a1, b1, threshold, t2, none);
+  }
+  cnt = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
   if (lane == 0) wsum[w] = cnt;
   __syncthreads();
   if (w == 0) {
-    const int t = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(wsum[lane])));
-    if (lane == 0) cta_sum[blockIdx.x] = t;
+    const int t = static_cast<int>(__reduce_add_sync(0xffffffffu, lane < kAggWarps ? wsum[lane] : 0u));
+    if (lane == 0) span_sum[blockIdx.x] = t;
   }
 }
 
-__global__ void __launch_bounds__(kAggRows * 32) compact_kernel(const uint8_t* __restrict__ mask, int64_t rows,
-                                                                int nb, const int32_t* __restrict__ row_cnt,
-                                                                const int32_t* __restrict__ cta_sum,
-                                                                int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap,
-                                                                int64_t* nnz_out, int* status) {
-  __shared__ long long wpart[kAggRows];
-  __shared__ int wcnt[kAggRows];
+template <bool kVec>
+__global__ void __launch_bounds__(kAggThreads) compact_kernel(const uint8_t* __restrict__ mask, int64_t cells,
+                                                              int nb, int64_t rows, int64_t span,
+                                                              const int32_t* __restrict__ span_sum,
+                                                              int32_t* __restrict__ row_ptr,
+                                                              int32_t* __restrict__ col_idx, int64_t nnz_cap,
+                                                              int64_t* nnz_out, int* status) {
+  __shared__ long long wbefore[kAggWarps];
+  __shared__ int wtot[2][kAggWarps];
+  __shared__ int32_t stage[kAggWarps][32 * kAggChunk];  // a warp's columns of one round
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // the kept blocks of every earlier CTA
+  // the kept cells of every earlier span
   long long before = 0;
-  for (int64_t i = threadIdx.x; i < blockIdx.x; i += blockDim.x) before += cta_sum[i];
+  for (int64_t i = threadIdx.x; i < blockIdx.x; i += kAggThreads) before += span_sum[i];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kAggRows + w;
-  const int cnt = row < rows ? row_cnt[row] : 0;
-  if (lane == 0) {
-    wpart[w] = before;
-    wcnt[w] = cnt;
-  }
+  if (lane == 0) wbefore[w] = before;
   __syncthreads();
-  // lane i of every warp takes warp i's partials
-  long long base = wpart[lane];
+  long long rank0 = 0;  // rank of the current round's first kept cell
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) base += __shfl_xor_sync(0xffffffffu, base, o);
-  const unsigned cw = static_cast<unsigned>(wcnt[lane]);
-  const long long mine = __reduce_add_sync(0xffffffffu, lane < w ? cw : 0u);
-  const long long total = __reduce_add_sync(0xffffffffu, cw);
-  long long pos = base + mine;  // this row's first entry
-  if (row < rows) {
-    if (lane == 0) row_ptr[row] = static_cast<int32_t>(pos);
-    const uint8_t* src = mask + row * nb;
-    for (int c0 = 0; c0 < nb; c0 += 32) {
-      const int c = c0 + lane;
-      const bool k = c < nb && src[c];
-      const uint32_t bal = __ballot_sync(0xffffffffu, k);
-      if (k) {
-        const int64_t at = pos + __popc(bal & ((1u << lane) - 1u));
-        if (at < nnz_cap) col_idx[at] = c;
-      }
-      pos += __popc(bal);
+  for (int i = 0; i < kAggWarps; ++i) rank0 += wbefore[i];
+  const int64_t s0 = static_cast<int64_t>(blockIdx.x) * span;
+  const int64_t s1 = s0 + span < cells ? s0 + span : cells;
+  // row and column of the lane's chunk start, advanced by one round per step
+  // (cells <= INT_MAX, so 32-bit flat indices)
+  const uint32_t unb = static_cast<uint32_t>(nb);
+  const uint32_t g0 = static_cast<uint32_t>(s0) + threadIdx.x * kAggChunk;
+  uint32_t row = g0 / unb;
+  int col = static_cast<int>(g0 - row * unb);
+  const uint32_t row_step = kAggRound / unb;
+  const int col_step = static_cast<int>(kAggRound % unb);
+  int buf = 0;
+  for (int64_t r0 = s0; r0 < s1; r0 += kAggRound, buf ^= 1) {  // uniform over the CTA
+    const int64_t g = r0 + threadIdx.x * kAggChunk;
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
+    if (kVec && g + kAggChunk <= s1) {
+      const uint4 v = *reinterpret_cast<const uint4*>(mask + g);
+      m[0] = v.x;
+      m[1] = v.y;
+      m[2] = v.z;
+      m[3] = v.w;
+    } else {
+      for (int j = 0; j < kAggChunk && g + j < s1; ++j)
+        m[j >> 2] |= static_cast<uint32_t>(mask[g + j] != 0) << (8 * (j & 3));
     }
+    const uint32_t bits = chunk_bits(m);
+    const int c = __popc(bits);
+    int inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
+    }
+    if (lane == 31) wtot[buf][w] = inc;
+    __syncthreads();  // wtot[buf] is rewritten two rounds later, after the next round's barrier
+    int wbase = 0, rtot = 0;
+#pragma unroll
+    for (int i = 0; i < kAggWarps; ++i) {
+      const int t = wtot[buf][i];
+      wbase += i < w ? t : 0;
+      rtot += t;
+    }
+    const long long wpos = rank0 + wbase;  // the warp's first rank this round
+    rank0 += rtot;
+    int at = inc - c;  // the lane's first slot in the warp's stage
+    if (g < s1) {
+      const int len = s1 - g < kAggChunk ? static_cast<int>(s1 - g) : kAggChunk;
+      // rows that start in the chunk: their first cell's rank
+      uint32_t rr = row + (col != 0 ? 1u : 0u);
+      for (int j = col != 0 ? nb - col : 0; j < len; j += nb, ++rr)
+        row_ptr[rr] = static_cast<int32_t>(wpos + at + __popc(bits & ((1u << j) - 1u)));
+      // kept cells only
+      for (uint32_t b = bits; b; b &= b - 1) {
+        int cc = col + __ffs(b) - 1;
+        while (cc >= nb) cc -= nb;
+        stage[w][at++] = cc;
+      }
+    }
+    col += col_step;
+    row += row_step;
+    if (col >= nb) {
+      col -= nb;
+      ++row;
+    }
+    __syncwarp();
+    // the warp's kept columns are one run of col_idx: coalesced stores
+    const int wcount = __shfl_sync(0xffffffffu, inc, 31);
+    for (int i = lane; i < wcount; i += 32)
+      if (wpos + i < nnz_cap) col_idx[wpos + i] = stage[w][i];
+    __syncwarp();
   }
   if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
-    const long long grand = base + total;
-    row_ptr[rows] = static_cast<int32_t>(grand);
-    *nnz_out = grand;
-    if (grand > nnz_cap) record_error(status, CALIBATT_ERR_CAPACITY);
+    row_ptr[rows] = static_cast<int32_t>(rank0);
+    *nnz_out = rank0;
+    if (rank0 > nnz_cap) record_error(status, CALIBATT_ERR_CAPACITY);
   }
 }
 
@@ -189,16 +295,29 @@ int launch_accumulate(const uint8_t* mask, int64_t cells, uint16_t* counts, cuda
 int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold, uint8_t* mask, int32_t* row_ptr,
                      int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* scratch, int* status,
                      cudaStream_t stream) {
-  const unsigned ctas = static_cast<unsigned>((rows + kAggRows - 1) / kAggRows);
-  int32_t* row_cnt = scratch;
-  int32_t* cta_sum = scratch + rows;
-  binarize_kernel<<<ctas, kAggRows * 32, 0, stream>>>(counts, rows, nb, threshold, mask, row_cnt, cta_sum);
-  compact_kernel<<<ctas, kAggRows * 32, 0, stream>>>(mask, rows, nb, row_cnt, cta_sum, row_ptr, col_idx, nnz_cap, nnz,
-                                                     status);
+  const int64_t cells = rows * nb;
+  // rounds per span: at least one row's worth of cells (so spans <= rows),
+  // else up to 4 while the grid still overfills the SMs
+  const int64_t by_row = (nb + kAggRound - 1) / kAggRound;
+  int64_t by_fill = (cells + kAggRound * kAggFill - 1) / (kAggRound * kAggFill);
+  if (by_fill > 4) by_fill = 4;
+  const int64_t span = (by_row > by_fill ? by_row : by_fill) * kAggRound;
+  const unsigned ctas = static_cast<unsigned>((cells + span - 1) / span);
+  const bool vec = ((reinterpret_cast<uintptr_t>(counts) | reinterpret_cast<uintptr_t>(mask)) & 15u) == 0;
+  if (vec) {
+    binarize_kernel<true><<<ctas, kAggThreads, 0, stream>>>(counts, cells, span, threshold, mask, scratch);
+    compact_kernel<true><<<ctas, kAggThreads, 0, stream>>>(mask, cells, nb, rows, span, scratch, row_ptr, col_idx,
+                                                           nnz_cap, nnz, status);
+  } else {
+    binarize_kernel<false><<<ctas, kAggThreads, 0, stream>>>(counts, cells, span, threshold, mask, scratch);
+    compact_kernel<false><<<ctas, kAggThreads, 0, stream>>>(mask, cells, nb, rows, span, scratch, row_ptr, col_idx,
+                                                            nnz_cap, nnz, status);
+  }
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
 }
 
-int64_t aggregate_scratch_ints(int64_t rows) { return rows + (rows + kAggRows - 1) / kAggRows; }
+// spans <= rows: a span holds at least nb cells
+int64_t aggregate_scratch_ints(int64_t rows) { return rows; }
 
 int launch_gather(const void* q, int n, int heads, const int32_t* rep_heads, int n_rep, int H, int W, int k_anchor,
                   const AnchorTable& tab, void* out, int* status, cudaStream_t stream) {

@@ -84,8 +84,8 @@ long long eps_to_fixed(double eps);
 int launch_select(const float* energy, int64_t rows, int nb, long long eps_fx, uint8_t* mask, int32_t* kept,
                   uint16_t* counts, uint8_t* tie, long long tie_fx, cudaStream_t stream);
 int launch_accumulate(const uint8_t* mask, int64_t cells, uint16_t* counts, cudaStream_t stream);
-// scratch: aggregate_scratch_ints(rows) int32 (per-row kept counts, then one
-// total per CTA of rows), every entry rewritten by each call
+// scratch: aggregate_scratch_ints(rows) int32 (one kept total per span of
+// the flat mask, at most one span per row), rewritten by each call
 int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold, uint8_t* mask, int32_t* row_ptr,
                      int32_t* col_idx, int64_t nnz_cap, int64_t* nnz, int32_t* scratch, int* status,
                      cudaStream_t stream);

@@ -18,10 +18,10 @@
 
 namespace calibatt {
 
-// One int32 per (head, block-row), at most CALIBATT_NOALLOC_MAX_ROWS rows,
-// then one per group of 32 rows: 1 MiB + 32 KiB. Every GPU that loads the
+// The aggregation's span totals: at most one int32 per (head, block-row), at
+// most CALIBATT_NOALLOC_MAX_ROWS rows: 1 MiB. Every GPU that loads the
 // library holds this array until exit.
-constexpr int64_t kNoallocScratchInts = CALIBATT_NOALLOC_MAX_ROWS + CALIBATT_NOALLOC_MAX_ROWS / 32;
+constexpr int64_t kNoallocScratchInts = CALIBATT_NOALLOC_MAX_ROWS;
 static __device__ __align__(256) int32_t g_noalloc_row_cnt[kNoallocScratchInts];
 
 namespace {

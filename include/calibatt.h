@@ -523,9 +523,9 @@ int calibatt_bank_get(const calibatt_bank* bank, int t, int l, calibatt_bank_ent
  * or a serving loop under a fixed memory budget where an allocation could fail
  * or stall. Same arguments, outputs and errors as calibatt_aggregate_masks
  * (the caller still passes counts, mask, row_ptr, col_idx and nnz); the
- * per-row counts (and one total per 32 rows) live in a static device array
- * of CALIBATT_NOALLOC_MAX_ROWS + CALIBATT_NOALLOC_MAX_ROWS / 32 int32
- * (1 MiB + 32 KiB), held by every GPU that loads the library until exit.
+ * aggregation's kept totals (one per span of the flat mask, at most one per
+ * row) live in a static device array of CALIBATT_NOALLOC_MAX_ROWS int32
+ * (1 MiB), held by every GPU that loads the library until exit.
  *  - Returns CALIBATT_ERR_ARG when heads * nb > CALIBATT_NOALLOC_MAX_ROWS.
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *  - The first call on a device looks up the array's device address (once per
@@ -533,7 +533,7 @@ int calibatt_bank_get(const calibatt_bank* bank, int t, int l, calibatt_bank_ent
  *    stream capture.
  *  - All calls share the array: calls whose kernels overlap on the GPU (for
  *    example on two streams at once) race and corrupt each other's results.
- *    Every count in it is rewritten by each call before it is read, so
+ *    Every total in it is rewritten by each call before it is read, so
  *    nothing needs clearing. */
 int calibatt_aggregate_masks_noalloc(const uint16_t* counts, int n_inputs, int heads, int nb, double rho,
                                      uint8_t* mask, int32_t* row_ptr, int32_t* col_idx, int64_t nnz_cap,

@@ -125,6 +125,48 @@ def test_accumulate_and_aggregate_match_oracle(oracle):
         assert int(nnz.item()) == int(m_ref.sum())
 
 
+@pytest.mark.parametrize("rows,cols", [(1, 1), (45, 591), (3, 20000), (2000, 37)])
+def test_aggregate_spans_ragged_tails_and_alignment(oracle, rows, cols):
+    """The aggregation walks the flat mask in spans of whole 4096-cell rounds
+    (at least one row each), with 16-byte vector accesses when counts and mask
+    are 16-byte aligned and byte accesses otherwise. Several spans, a ragged
+    last span, rows wider than the default span, and both access forms give
+    the oracle's mask and skip list bit for bit."""
+    binding = require_gpu()
+    lib = binding.load()
+    rng = np.random.default_rng(rows * 7 + cols)
+    n_in = 5
+    masks = (rng.random((n_in, rows, cols)) < rng.random((1, rows, 1))).astype(np.uint8)
+    m_ref, c_ref = oracle.aggregate(masks, 0.5)
+    rp_ref, ci_ref = oracle.mask_rows_to_csr(m_ref[None])
+    dev = torch.device("cuda")
+    cells = rows * cols
+    for c_off, m_off in ((0, 0), (1, 3)):  # element / byte offsets into the buffers
+        cbuf = torch.zeros(cells + 8, dtype=torch.uint16, device=dev)
+        cbuf[c_off:c_off + cells] = torch.from_numpy(c_ref.astype(np.uint16).reshape(-1)).to(dev)
+        mbuf = torch.full((cells + 16,), 7, dtype=torch.uint8, device=dev)
+        row_ptr = torch.full((rows + 1,), -1, dtype=torch.int32, device=dev)
+        col_idx = torch.full((cells,), -1, dtype=torch.int32, device=dev)
+        nnz = torch.zeros(1, dtype=torch.int64, device=dev)
+        ws = torch.empty(lib.calibatt_aggregate_rows_workspace_size(rows), dtype=torch.uint8, device=dev)
+        rc = lib.calibatt_aggregate_mask_rows(cbuf.data_ptr() + 2 * c_off, n_in, rows, cols, 0.5,
+                                              mbuf.data_ptr() + m_off, binding._ptr(row_ptr),
+                                              binding._ptr(col_idx), cells, binding._ptr(nnz), binding._ptr(ws),
+                                              ws.numel(), binding._stream(None))
+        assert rc == 0
+        torch.cuda.synchronize()
+        assert binding.get_status() == 0
+        mb = mbuf.cpu().numpy()
+        np.testing.assert_array_equal(mb[m_off:m_off + cells].reshape(rows, cols), m_ref)
+        assert np.all(mb[:m_off] == 7) and np.all(mb[m_off + cells:] == 7)  # nothing written outside
+        total = int(nnz.item())
+        assert total == int(m_ref.sum())
+        np.testing.assert_array_equal(row_ptr.cpu().numpy(), rp_ref)
+        ci = col_idx.cpu().numpy()
+        np.testing.assert_array_equal(ci[:total], ci_ref)
+        assert np.all(ci[total:] == -1)
+
+
 def test_aggregate_capacity_is_reported():
     binding = require_gpu()
     dev = torch.device("cuda")
