@@ -80,9 +80,11 @@ __device__ __forceinline__ uint32_t chunk_bits(const uint32_t (&m)[4]) {
   return bits;
 }
 
+// Flat indices, ranks and spans fit in 32 bits (cells <= INT_MAX, a span at
+// most cells + one round), which keeps the index arithmetic single-word.
 template <bool kVec>
 __device__ __forceinline__ int binarize_chunk(const uint16_t* __restrict__ counts, uint8_t* __restrict__ mask,
-                                              int64_t g, int64_t s1, const uint4& a, const uint4& b, int threshold,
+                                              uint32_t g, uint32_t s1, const uint4& a, const uint4& b, int threshold,
                                               uint32_t t2, bool none) {
   if (kVec && g + kAggChunk <= s1) {
     uint4 m;
@@ -94,7 +96,7 @@ __device__ __forceinline__ int binarize_chunk(const uint16_t* __restrict__ count
     return __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
   }
   int cnt = 0;
-  for (int j = 0; j < kAggChunk && g + j < s1; ++j) {
+  for (uint32_t j = 0; j < kAggChunk && g + j < s1; ++j) {
     const int k = counts[g + j] >= threshold ? 1 : 0;
     mask[g + j] = static_cast<uint8_t>(k);
     cnt += k;
@@ -103,20 +105,20 @@ __device__ __forceinline__ int binarize_chunk(const uint16_t* __restrict__ count
 }
 
 template <bool kVec>
-__global__ void __launch_bounds__(kAggThreads) binarize_kernel(const uint16_t* __restrict__ counts, int64_t cells,
-                                                               int64_t span, int threshold,
+__global__ void __launch_bounds__(kAggThreads) binarize_kernel(const uint16_t* __restrict__ counts, uint32_t cells,
+                                                               uint32_t span, int threshold,
                                                                uint8_t* __restrict__ mask,
                                                                int32_t* __restrict__ span_sum) {
   __shared__ int wsum[kAggWarps];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t s0 = static_cast<int64_t>(blockIdx.x) * span;
-  const int64_t s1 = s0 + span < cells ? s0 + span : cells;
+  const uint32_t s0 = blockIdx.x * span;
+  const uint32_t s1 = cells - s0 > span ? s0 + span : cells;
   const bool none = threshold > 65535;  // counts are 16-bit
   const uint32_t t2 = static_cast<uint32_t>(threshold > 0 ? threshold : 0) * 0x10001u;
   int cnt = 0;
   // two rounds per step, both rounds' loads in flight before either is used
-  for (int64_t g = s0 + threadIdx.x * kAggChunk; g < s1; g += 2 * kAggRound) {
-    const int64_t h = g + kAggRound;
+  for (uint32_t g = s0 + threadIdx.x * kAggChunk; g < s1; g += 2 * kAggRound) {
+    const uint32_t h = g + kAggRound;
     uint4 a0 = {}, b0 = {}, a1 = {}, b1 = {};
     if (kVec && g + kAggChunk <= s1) {
       a0 = *reinterpret_cast<const uint4*>(counts + g);
@@ -139,39 +141,38 @@ __global__ void __launch_bounds__(kAggThreads) binarize_kernel(const uint16_t* _
 }
 
 template <bool kVec>
-__global__ void __launch_bounds__(kAggThreads) compact_kernel(const uint8_t* __restrict__ mask, int64_t cells,
-                                                              int nb, int64_t rows, int64_t span,
+__global__ void __launch_bounds__(kAggThreads) compact_kernel(const uint8_t* __restrict__ mask, uint32_t cells,
+                                                              int nb, uint32_t rows, uint32_t span,
                                                               const int32_t* __restrict__ span_sum,
                                                               int32_t* __restrict__ row_ptr,
                                                               int32_t* __restrict__ col_idx, int64_t nnz_cap,
                                                               int64_t* nnz_out, int* status) {
-  __shared__ long long wbefore[kAggWarps];
+  __shared__ int wbefore[kAggWarps];
   __shared__ int wtot[2][kAggWarps];
   __shared__ int32_t stage[kAggWarps][32 * kAggChunk];  // a warp's columns of one round
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cap = nnz_cap < cells ? static_cast<int>(nnz_cap) : static_cast<int>(cells);  // ranks < cells
   // the kept cells of every earlier span
-  long long before = 0;
-  for (int64_t i = threadIdx.x; i < blockIdx.x; i += kAggThreads) before += span_sum[i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+  int before = 0;
+  for (uint32_t i = threadIdx.x; i < blockIdx.x; i += kAggThreads) before += span_sum[i];
+  before = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(before)));
   if (lane == 0) wbefore[w] = before;
   __syncthreads();
-  long long rank0 = 0;  // rank of the current round's first kept cell
+  int rank0 = 0;  // rank of the current round's first kept cell
 #pragma unroll
   for (int i = 0; i < kAggWarps; ++i) rank0 += wbefore[i];
-  const int64_t s0 = static_cast<int64_t>(blockIdx.x) * span;
-  const int64_t s1 = s0 + span < cells ? s0 + span : cells;
+  const uint32_t s0 = blockIdx.x * span;
+  const uint32_t s1 = cells - s0 > span ? s0 + span : cells;
   // row and column of the lane's chunk start, advanced by one round per step
-  // (cells <= INT_MAX, so 32-bit flat indices)
   const uint32_t unb = static_cast<uint32_t>(nb);
-  const uint32_t g0 = static_cast<uint32_t>(s0) + threadIdx.x * kAggChunk;
+  const uint32_t g0 = s0 + threadIdx.x * kAggChunk;
   uint32_t row = g0 / unb;
   int col = static_cast<int>(g0 - row * unb);
   const uint32_t row_step = kAggRound / unb;
   const int col_step = static_cast<int>(kAggRound % unb);
+  int32_t* const my_stage = stage[w];
   int buf = 0;
-  for (int64_t r0 = s0; r0 < s1; r0 += kAggRound, buf ^= 1) {  // uniform over the CTA
-    const int64_t g = r0 + threadIdx.x * kAggChunk;
+  for (uint32_t g = g0; g - threadIdx.x * kAggChunk < s1; g += kAggRound, buf ^= 1) {  // uniform over the CTA
     uint32_t m[4] = {0u, 0u, 0u, 0u};
     if (kVec && g + kAggChunk <= s1) {
       const uint4 v = *reinterpret_cast<const uint4*>(mask + g);
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kAggThreads) compact_kernel(const uint8_t* __r
       m[2] = v.z;
       m[3] = v.w;
     } else {
-      for (int j = 0; j < kAggChunk && g + j < s1; ++j)
+      for (uint32_t j = 0; j < kAggChunk && g + j < s1; ++j)
         m[j >> 2] |= static_cast<uint32_t>(mask[g + j] != 0) << (8 * (j & 3));
     }
     const uint32_t bits = chunk_bits(m);
@@ -200,20 +201,26 @@ __global__ void __launch_bounds__(kAggThreads) compact_kernel(const uint8_t* __r
       wbase += i < w ? t : 0;
       rtot += t;
     }
-    const long long wpos = rank0 + wbase;  // the warp's first rank this round
+    const int wpos = rank0 + wbase;  // the warp's first rank this round
     rank0 += rtot;
     int at = inc - c;  // the lane's first slot in the warp's stage
     if (g < s1) {
       const int len = s1 - g < kAggChunk ? static_cast<int>(s1 - g) : kAggChunk;
-      // rows that start in the chunk: their first cell's rank
-      uint32_t rr = row + (col != 0 ? 1u : 0u);
-      for (int j = col != 0 ? nb - col : 0; j < len; j += nb, ++rr)
-        row_ptr[rr] = static_cast<int32_t>(wpos + at + __popc(bits & ((1u << j) - 1u)));
-      // kept cells only
-      for (uint32_t b = bits; b; b &= b - 1) {
-        int cc = col + __ffs(b) - 1;
-        while (cc >= nb) cc -= nb;
-        stage[w][at++] = cc;
+      if (col + len <= nb) {  // the chunk lies in one row
+        if (col == 0) row_ptr[row] = wpos + at;
+#pragma unroll
+        for (int j = 0; j < kAggChunk; ++j)
+          if ((bits >> j) & 1u) my_stage[at++] = col + j;
+      } else {
+        // rows that start in the chunk: their first cell's rank
+        uint32_t rr = row + (col != 0 ? 1u : 0u);
+        for (int j = col != 0 ? nb - col : 0; j < len; j += nb, ++rr)
+          row_ptr[rr] = wpos + at + __popc(bits & ((1u << j) - 1u));
+        for (uint32_t b = bits; b; b &= b - 1) {
+          int cc = col + __ffs(b) - 1;
+          while (cc >= nb) cc -= nb;
+          my_stage[at++] = cc;
+        }
       }
     }
     col += col_step;
@@ -225,12 +232,12 @@ __global__ void __launch_bounds__(kAggThreads) compact_kernel(const uint8_t* __r
     __syncwarp();
     // the warp's kept columns are one run of col_idx: coalesced stores
     const int wcount = __shfl_sync(0xffffffffu, inc, 31);
-    for (int i = lane; i < wcount; i += 32)
-      if (wpos + i < nnz_cap) col_idx[wpos + i] = stage[w][i];
+    const int lim = cap - wpos < wcount ? cap - wpos : wcount;
+    for (int i = lane; i < lim; i += 32) col_idx[wpos + i] = my_stage[i];
     __syncwarp();
   }
   if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
-    row_ptr[rows] = static_cast<int32_t>(rank0);
+    row_ptr[rows] = rank0;
     *nnz_out = rank0;
     if (rank0 > nnz_cap) record_error(status, CALIBATT_ERR_CAPACITY);
   }
@@ -304,13 +311,16 @@ int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold
   const int64_t span = (by_row > by_fill ? by_row : by_fill) * kAggRound;
   const unsigned ctas = static_cast<unsigned>((cells + span - 1) / span);
   const bool vec = ((reinterpret_cast<uintptr_t>(counts) | reinterpret_cast<uintptr_t>(mask)) & 15u) == 0;
+  // cells <= INT_MAX (checked by every caller): 32-bit flat indices
+  const uint32_t c32 = static_cast<uint32_t>(cells), s32 = static_cast<uint32_t>(span);
+  const uint32_t r32 = static_cast<uint32_t>(rows);
   if (vec) {
-    binarize_kernel<true><<<ctas, kAggThreads, 0, stream>>>(counts, cells, span, threshold, mask, scratch);
-    compact_kernel<true><<<ctas, kAggThreads, 0, stream>>>(mask, cells, nb, rows, span, scratch, row_ptr, col_idx,
+    binarize_kernel<true><<<ctas, kAggThreads, 0, stream>>>(counts, c32, s32, threshold, mask, scratch);
+    compact_kernel<true><<<ctas, kAggThreads, 0, stream>>>(mask, c32, nb, r32, s32, scratch, row_ptr, col_idx,
                                                            nnz_cap, nnz, status);
   } else {
-    binarize_kernel<false><<<ctas, kAggThreads, 0, stream>>>(counts, cells, span, threshold, mask, scratch);
-    compact_kernel<false><<<ctas, kAggThreads, 0, stream>>>(mask, cells, nb, rows, span, scratch, row_ptr, col_idx,
+    binarize_kernel<false><<<ctas, kAggThreads, 0, stream>>>(counts, c32, s32, threshold, mask, scratch);
+    compact_kernel<false><<<ctas, kAggThreads, 0, stream>>>(mask, c32, nb, r32, s32, scratch, row_ptr, col_idx,
                                                             nnz_cap, nnz, status);
   }
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
