@@ -19,11 +19,13 @@ namespace calibatt {
 // One warp per block-row of energies, four rows per CTA, each warp with 128
 // bytes of shared scratch; no block barriers. PER (columns per lane, >= nb / 32)
 // sizes the per-lane register arrays. Lanes read and write the row's columns
-// interleaved (column lane + 32 i), so every access is coalesced.
+// interleaved (column lane + 32 i), so every access is coalesced. The launch
+// bounds hold the register count at 80 (96 for PER = 32) without spills, so
+// that 6 (5) CTAs share an SM: the search's warp-sum chains need the warps.
 template <int PER>
-__global__ void __launch_bounds__(128) select_kernel(const float* __restrict__ energy, int64_t rows, int nb,
-                                                     long long eps_fx, uint8_t* mask, int32_t* kept,
-                                                     uint16_t* counts, uint8_t* tie, long long tie_fx) {
+__global__ void __launch_bounds__(128, PER <= 24 ? 6 : 5)
+    select_kernel(const float* __restrict__ energy, int64_t rows, int nb, long long eps_fx, uint8_t* mask,
+                  int32_t* kept, uint16_t* counts, uint8_t* tie, long long tie_fx) {
   __shared__ __align__(16) float scratch[4][kSelectScratchBytes / 4];
   const int w = threadIdx.x >> 5;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + w;
