@@ -557,8 +557,13 @@ def calibration_kernels(binding, wl, q, k, dev, stream, pk):
     annz = torch.zeros(1, dtype=torch.int64, device=dev)
     lib = binding.load()
 
+    # the aggregation's input: this input's eps = 0.9 selection as the counts
+    # of one input (kept where the mask is), so the skip list has ~19 % of the
+    # blocks
+    acounts = cmask.to(torch.int16).view(torch.uint16)
+
     def agg_call():
-        lib.calibatt_aggregate_masks(binding._ptr(ccounts), 64, heads, nb, 0.5, binding._ptr(am),
+        lib.calibatt_aggregate_masks(binding._ptr(acounts), 1, heads, nb, 0.5, binding._ptr(am),
                                      binding._ptr(arp), binding._ptr(aci), aci.numel(), binding._ptr(annz),
                                      binding._ptr(agg_ws), agg_ws.numel(),
                                      binding._stream(torch.cuda.current_stream()))
@@ -593,6 +598,7 @@ def calibration_kernels(binding, wl, q, k, dev, stream, pk):
         "select_ms": s_ms, "select_gbs": sel_bytes / (s_ms * 1e-3) / 1e9,
         "select_bytes": sel_bytes,
         "aggregate_ms": a_ms, "aggregate_gbs": agg_bytes / (a_ms * 1e-3) / 1e9, "aggregate_bytes": agg_bytes,
+        "aggregate_kept_blocks": kept_agg,
         "eps": 0.9, "kept_fraction_at_eps": float(cmask.float().mean().item()),
         "tie_affected_rows_at_eps": int(tie.sum().item()),
         "pixel_row_energy_ms": p_ms, "pixel_row_energy_tflops_issued": 2 * f_alg / (p_ms * 1e-3) / 1e12,

@@ -708,7 +708,7 @@ size_t calibatt_energy_workspace_size(int heads, int n) {
   const int64_t nb = (static_cast<int64_t>(n) + 127) / 128;
   const int64_t units = heads * nb;
   if (units > INT_MAX / 2 || nb > CALIBATT_MAX_CALIB_NB) return 0;
-  const size_t bytes = static_cast<size_t>(2 * score_grid(static_cast<int>(units))) * nb * 128 * sizeof(float2);
+  const size_t bytes = static_cast<size_t>(energy_ws_floats(2 * score_grid(static_cast<int>(units)), nb)) * sizeof(float);
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
@@ -735,7 +735,7 @@ int calibatt_block_energy_1pass(const calibatt_bf16* q, const calibatt_bf16* k, 
   p.n_units = heads * nb;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_out = n;
-  p.energy_ws = static_cast<float2*>(ws);
+  p.energy_ws = static_cast<float*>(ws);
   p.energy = energy;
   p.fuse_select = fuse_select ? 1 : 0;
   p.eps_fx = eps_to_fixed(eps);
@@ -863,7 +863,7 @@ size_t calibatt_anchor_energy_workspace_size(int heads, int n_rep, int frames, i
   const int64_t units = n_rep * anchor_blocks(frames, W, k_anchor);
   if (n > INT_MAX / 2 || units > INT_MAX / 2 || nb > CALIBATT_MAX_CALIB_NB) return 0;
   const size_t packed = calibatt_repeat_workspace_size(n_rep, frames, H, W, k_anchor);
-  const size_t energy = static_cast<size_t>(2 * score_grid(static_cast<int>(units))) * nb * 128 * sizeof(float2);
+  const size_t energy = static_cast<size_t>(energy_ws_floats(2 * score_grid(static_cast<int>(units)), nb)) * sizeof(float);
   return packed + ((energy + 255) & ~static_cast<size_t>(255));
 }
 
@@ -911,7 +911,7 @@ int calibatt_anchor_block_energy(const calibatt_bf16* q, const calibatt_bf16* k,
   p.n_units = n_rep * p.nbq;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_out = n;
-  p.energy_ws = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + packed);
+  p.energy_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + packed);
   p.energy = energy;
   p.fuse_select = fuse_select ? 1 : 0;
   p.eps_fx = eps_to_fixed(eps);

@@ -10,6 +10,13 @@ namespace calibatt {
 constexpr int kMaxAnchors = 64;
 
 // Parameters of the persistent tensor-core attention kernel (all modes).
+// Key blocks per chunk of the single-pass energy workspace.
+constexpr int kEnergyChunk = 8;
+// fp32 words of that workspace for `slots` query tiles of nb key blocks.
+inline int64_t energy_ws_floats(int64_t slots, int64_t nb) {
+  return slots * ((nb + kEnergyChunk - 1) / kEnergyChunk) * (kEnergyChunk + 1) * 128;
+}
+
 struct KernelParams {
   int n_q;        // query rows per head in the Q tensor
   int n_k;        // key rows per head
@@ -55,8 +62,10 @@ struct KernelParams {
   float* pix_energy;   // [heads_q][pix_rows][nbk] or NULL
   int pix_W, pix_rows;
   float pix_inv_W;
-  // single-pass energy: per slot, per key block, per row (tile sum, running max)
-  float2* energy_ws;   // [2 * grid][nbk][128]
+  // single-pass energy: per slot, per chunk of kEnergyChunk key blocks, per
+  // row: the chunk's tile sums relative to the row's running max at the
+  // chunk's end, then that max
+  float* energy_ws;    // [2 * grid][ceil(nbk / kEnergyChunk)][kEnergyChunk + 1][128]
   int* status;         // device status word
   uint64_t wait_limit_ns;  // limit of the pipeline's bounded waits
 };

@@ -5,11 +5,13 @@
 //   kEnergy:  second pass: per tile, sum_ij 2^(scale' S_ij - lse_i) -> E[r][c],
 //             then the greedy eps selection of the finished row (select.cuh)
 //   kEnergy1: the same energies in one pass: each row keeps its exact
-//             running max m and sum l, and stores every tile's sum t relative
-//             to m (with m) in a workspace; when the row is done,
-//             t * 2^(m - lse) gives its share of E[r][c] exactly as the second
-//             pass would, and the row's tiles are reduced and selected as
-//             above. S is computed once instead of twice.
+//             running max m and sum l, and stores every tile's sum t in a
+//             workspace, chunks of 8 tiles relative to the m reached at the
+//             chunk's end (when m grows, the chunk's stored sums are rescaled
+//             with l), that m after them (36 bytes per 8 tiles); when the
+//             row is done, t * 2^(m - lse) gives its share of E[r][c] as the
+//             second pass would, and the row's tiles are reduced and selected
+//             as above. S is computed once instead of twice.
 //
 // CTA (320 threads, one per SM): two query-tile slots; warps 0-3 and 4-7 are
 // the slots' row warpgroups (thread = query row = TMEM lane), warp 8 loads Q
@@ -266,6 +268,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         pix_hq = u.hq;
       }
       float m_run = -INFINITY, l_run = 0.f;
+      // single pass: this row's words of the chunk holding key block j
+      const int64_t n_chunks = (p.nbk + kEnergyChunk - 1) / kEnergyChunk;
+      auto chunk_ws = [&](int j) {
+        return p.energy_ws + ((static_cast<int64_t>(g) * n_chunks + j / kEnergyChunk) * (kEnergyChunk + 1)) * 128 + row;
+      };
       for (int j = 0; j < u.nnz; ++j) {
         const int buf = n_sfull & 1;
         float acc = 0.f;
@@ -288,7 +295,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           if (MODE == kLse || MODE == kEnergy1) {
             const float mx = row_max128(sv) * p.scale_log2;
             const float m_new = fmaxf(m_run, mx);
-            if (m_run != -INFINITY) l_run *= ex2_approx(m_run - m_new);
+            if (m_new > m_run && m_run != -INFINITY) {  // 2^0 = 1 exactly: no change to skip
+              const float f = ex2_approx(m_run - m_new);
+              l_run *= f;
+              if (MODE == kEnergy1) {
+                // the chunk's sums stored so far follow the new max (rare:
+                // a row's max grows a few times, mostly in its first tiles)
+                float* w = chunk_ws(j);
+                for (int i = 0; i < j % kEnergyChunk; ++i) w[i * 128] *= f;
+              }
+            }
             m_run = m_new;
             ref = m_new;
           } else {
@@ -312,9 +328,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             acc = (s01.x + s01.y) + (s23.x + s23.y);
           }
           if (MODE != kEnergy) l_run += acc;
-          // single pass: keep the tile's sum relative to the running max
-          if (MODE == kEnergy1)
-            p.energy_ws[(static_cast<int64_t>(g) * p.nbk + j) * 128 + row] = make_float2(acc, m_run);
+          // single pass: store the tile's sum relative to the running max,
+          // and at the chunk's end that max
+          if (MODE == kEnergy1) {
+            const int slot = j % kEnergyChunk;
+            float* w = chunk_ws(j);
+            w[slot * 128] = acc;
+            if (slot == kEnergyChunk - 1 || j == u.nnz - 1) w[kEnergyChunk * 128] = m_run;
+          }
         }
         if (MODE == kEnergy && p.pix_energy) pix_add(acc, j);
         if (MODE == kEnergy) {
@@ -328,21 +349,18 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         if (ok) p.lse_ws[static_cast<int64_t>(u.hq) * p.nbq * 128 + qrow] = m_run + log2f(l_run);
       } else {
         if (MODE == kEnergy1) {
-          // every tile sum rescaled to the row's final log-sum-exp, then
-          // summed over the warp's 32 rows, eight key blocks at a time
+          // every chunk's tile sums rescaled to the row's final
+          // log-sum-exp, then summed over the warp's 32 rows
+          static_assert(kEnergyChunk == 8, "the reduction below takes eight key blocks at a time");
           const float lse_r = m_run + log2f(l_run);
-          const float2* wsr = p.energy_ws + static_cast<int64_t>(g) * p.nbk * 128 + row;
+          const float* wsr = p.energy_ws + static_cast<int64_t>(g) * n_chunks * (kEnergyChunk + 1) * 128 + row;
           for (int c0 = 0; c0 < p.nbk; c0 += 8) {
+            const float* wc = wsr + static_cast<int64_t>(c0 / 8) * (kEnergyChunk + 1) * 128;
+            const bool live = ok && row_valid;
+            const float sc = live ? ex2_approx(wc[kEnergyChunk * 128] - lse_r) : 0.f;
             float v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float x = 0.f;
-              if (ok && row_valid && c0 + i < p.nbk) {
-                const float2 w = wsr[static_cast<int64_t>(c0 + i) * 128];
-                x = w.x * ex2_approx(w.y - lse_r);
-              }
-              v[i] = x;
-            }
+            for (int i = 0; i < 8; ++i) v[i] = live && c0 + i < p.nbk ? wc[i * 128] * sc : 0.f;
             if (p.pix_energy) {
 #pragma unroll
               for (int i = 0; i < 8; ++i)

@@ -317,9 +317,11 @@ int calibatt_block_energy(const calibatt_bf16* q, const calibatt_bf16* k, int he
 size_t calibatt_energy_workspace_size(int heads, int n);
 
 /* calibatt_block_energy in one pass over the keys instead of two: each query
- * row keeps its exact running max m and running sum, and stores every key
- * block's sum of 2^(scale' s - m) with m in ws; once the row's log-sum-exp
- * is known the stored sums are rescaled and reduced into the same energies
+ * row keeps its exact running max m and running sum, and stores its key
+ * blocks' sums of 2^(scale' s - m) in ws, eight key blocks at a time, all
+ * relative to the m reached at the eighth (36 bytes per row and eight key
+ * blocks); once the row's log-sum-exp is known the stored sums are rescaled
+ * and reduced into the same energies
  * (and fused selection) as calibatt_block_energy, which computes S twice.
  * With pix_energy != NULL it also writes the profiles of
  * calibatt_pixel_row_energy for pixel rows of pix_W consecutive queries
