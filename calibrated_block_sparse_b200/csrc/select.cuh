@@ -162,6 +162,7 @@ __device__ __forceinline__ void warp_select(const float* E, int nb, long long ep
 
   uint32_t tau = 0;
   long long above = 0;  // sum of fx over blocks with energy > tau
+  int eq_count = -1;    // blocks with energy == tau, when the finish knows it
   if (mode == 2) {
     // prefix range [plo, phi] of tau's bit pattern, narrowed digit by digit
     // (bits 30..20, then 19..10, then 9..0) by binary search with fp32 sums,
@@ -235,6 +236,7 @@ __device__ __forceinline__ void warp_select(const float* E, int nb, long long ep
         const bool ok = lane < m && base + T >= eps_fx;
         tau = __reduce_max_sync(0xffffffffu, ok ? cb : 0u);
         above = base + warp_sum64(lane < m && cb > tau ? cf : 0);
+        eq_count = __popc(__ballot_sync(0xffffffffu, lane < m && cb == tau));  // tau's blocks are all candidates
       }
     } else if (plo == phi) {
       // more than 32 blocks with one energy: all candidates are equal
@@ -243,6 +245,7 @@ __device__ __forceinline__ void warp_select(const float* E, int nb, long long ep
         exact = true;
         tau = plo;
         above = base;
+        eq_count = m;
       }
     }
     if (!exact) tau = exact_cut_search<PER>(bits, top_bits, eps_fx, above);
@@ -271,20 +274,27 @@ __device__ __forceinline__ void warp_select(const float* E, int nb, long long ep
     while (r_need > 1 && (r_need - 1) * ft >= rem) --r_need;
     while (r_need * ft < rem) ++r_need;
   }
-  int before = 0;  // equal blocks in earlier columns
+  // every block equal to tau is kept when the cut needs all of them (the
+  // common case: one such block): no ranks among them are needed
+  const bool all_eq = mode == 2 && eq_count >= 0 && eq_count <= r_need;
+  int before = all_eq ? eq_count : 0;  // equal blocks in earlier columns (after the loop: all of them)
   int kept_mine = 0;
   uint32_t nxt = 0;  // largest energy below tau, plus one (0: none)
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int c = lane + 32 * i;
     const bool in = c < nb;
-    const bool eq = mode == 2 && in && bits[i] == tau;
-    const unsigned bal = __ballot_sync(0xffffffffu, eq);
     bool k;
-    if (mode == 0) k = in && c == top_col;
-    else if (mode == 1) k = in && bits[i] > 0;
-    else k = in && (bits[i] > tau || (eq && before + __popc(bal & lt_mask) < r_need));
-    before += __popc(bal);
+    if (all_eq) {
+      k = in && bits[i] >= tau;
+    } else {
+      const bool eq = mode == 2 && in && bits[i] == tau;
+      const unsigned bal = __ballot_sync(0xffffffffu, eq);
+      if (mode == 0) k = in && c == top_col;
+      else if (mode == 1) k = in && bits[i] > 0;
+      else k = in && (bits[i] > tau || (eq && before + __popc(bal & lt_mask) < r_need));
+      before += __popc(bal);
+    }
     kept_mine += k;
     if (in && bits[i] < tau && bits[i] + 1 > nxt) nxt = bits[i] + 1;
     if (in) {
