@@ -66,8 +66,8 @@ extern "C" int calibatt_aggregate_masks_noalloc(const uint16_t* counts, int n_in
   if (!scratch || !status) return CALIBATT_ERR_CUDA;
   int32_t thr = 0;
   calibatt_rho_threshold(n_inputs, rho, &thr);
-  // The first pass writes every per-row count and per-group total that the
-  // second reads, so the array needs no clearing between calls.
+  // The first pass writes every span total that the second reads, so the
+  // array needs no clearing between calls.
   return launch_aggregate(counts, rows, nb, thr, mask, row_ptr, col_idx, nnz_cap, nnz, scratch, status,
                           reinterpret_cast<cudaStream_t>(stream));
 }
