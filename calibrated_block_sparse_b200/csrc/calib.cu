@@ -56,6 +56,9 @@ __global__ void accumulate_kernel(const uint8_t* __restrict__ mask, int64_t cell
 //     kAggChunk cells ranked by a block scan per round; each warp stages its
 //     kept columns in shared memory and stores them as one coalesced run.
 //     The last CTA writes the grand total.
+// Above kPrefixSpans spans a one-CTA scan turns the totals into exclusive
+// prefixes between the two launches, so that a compaction CTA reads its
+// first rank instead of adding up every earlier span.
 // A span is a whole number of rounds, so with 16-byte aligned arrays every
 // lane chunk is one 16-byte mask vector and two 16-byte count vectors.
 // Scratch: one total per span.
@@ -142,21 +145,65 @@ __global__ void __launch_bounds__(kAggThreads) binarize_kernel(const uint16_t* _
   }
 }
 
+// Large grids: the span totals become exclusive prefixes in place (one CTA,
+// each thread a run of consecutive spans), so that a compaction CTA reads its
+// first rank instead of adding up every earlier span (quadratic in spans).
+constexpr int kScanThreads = 1024;
+constexpr unsigned kPrefixSpans = 4096;  // above this many spans the totals are scanned first
+
+__global__ void __launch_bounds__(kScanThreads) scan_spans_kernel(int32_t* span_sum, uint32_t spans) {
+  __shared__ int wpart[kScanThreads / 32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t per = (spans + kScanThreads - 1) / kScanThreads;
+  const uint32_t a = threadIdx.x * per;
+  const uint32_t b = a + per < spans ? a + per : spans;
+  int mine = 0;
+  for (uint32_t i = a; i < b; ++i) mine += span_sum[i];
+  int inc = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  if (lane == 31) wpart[w] = inc;
+  __syncthreads();
+  if (w == 0) {
+    int v = wpart[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += t;
+    }
+    wpart[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  int run = (w > 0 ? wpart[w - 1] : 0) + inc - mine;  // exclusive prefix of this thread's run
+  for (uint32_t i = a; i < b; ++i) {
+    const int t = span_sum[i];
+    span_sum[i] = run;
+    run += t;
+  }
+}
+
 template <bool kVec>
 __global__ void __launch_bounds__(kAggThreads) compact_kernel(const uint8_t* __restrict__ mask, uint32_t cells,
                                                               int nb, uint32_t rows, uint32_t span,
                                                               const int32_t* __restrict__ span_sum,
                                                               int32_t* __restrict__ row_ptr,
                                                               int32_t* __restrict__ col_idx, int64_t nnz_cap,
-                                                              int64_t* nnz_out, int* status) {
+                                                              int64_t* nnz_out, int* status, bool prefixed) {
   __shared__ int wbefore[kAggWarps];
   __shared__ int wtot[2][kAggWarps];
   __shared__ int32_t stage[kAggWarps][32 * kAggChunk];  // a warp's columns of one round
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cap = nnz_cap < cells ? static_cast<int>(nnz_cap) : static_cast<int>(cells);  // ranks < cells
-  // the kept cells of every earlier span
+  // the kept cells of every earlier span (already summed when prefixed)
   int before = 0;
-  for (uint32_t i = threadIdx.x; i < blockIdx.x; i += kAggThreads) before += span_sum[i];
+  if (prefixed) {
+    if (threadIdx.x == 0) before = span_sum[blockIdx.x];
+  } else {
+    for (uint32_t i = threadIdx.x; i < blockIdx.x; i += kAggThreads) before += span_sum[i];
+  }
   before = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(before)));
   if (lane == 0) wbefore[w] = before;
   __syncthreads();
@@ -316,14 +363,17 @@ int launch_aggregate(const uint16_t* counts, int64_t rows, int nb, int threshold
   // cells <= INT_MAX (checked by every caller): 32-bit flat indices
   const uint32_t c32 = static_cast<uint32_t>(cells), s32 = static_cast<uint32_t>(span);
   const uint32_t r32 = static_cast<uint32_t>(rows);
+  const bool prefixed = ctas > kPrefixSpans;
   if (vec) {
     binarize_kernel<true><<<ctas, kAggThreads, 0, stream>>>(counts, c32, s32, threshold, mask, scratch);
+    if (prefixed) scan_spans_kernel<<<1, kScanThreads, 0, stream>>>(scratch, ctas);
     compact_kernel<true><<<ctas, kAggThreads, 0, stream>>>(mask, c32, nb, r32, s32, scratch, row_ptr, col_idx,
-                                                           nnz_cap, nnz, status);
+                                                           nnz_cap, nnz, status, prefixed);
   } else {
     binarize_kernel<false><<<ctas, kAggThreads, 0, stream>>>(counts, c32, s32, threshold, mask, scratch);
+    if (prefixed) scan_spans_kernel<<<1, kScanThreads, 0, stream>>>(scratch, ctas);
     compact_kernel<false><<<ctas, kAggThreads, 0, stream>>>(mask, c32, nb, r32, s32, scratch, row_ptr, col_idx,
-                                                            nnz_cap, nnz, status);
+                                                            nnz_cap, nnz, status, prefixed);
   }
   return cudaGetLastError() == cudaSuccess ? CALIBATT_OK : CALIBATT_ERR_CUDA;
 }

@@ -167,6 +167,42 @@ def test_aggregate_spans_ragged_tails_and_alignment(oracle, rows, cols):
         assert np.all(ci[total:] == -1)
 
 
+def test_aggregate_scanned_span_prefixes(oracle):
+    """Above 4096 spans the span totals are scanned into prefixes by a third
+    launch before the compaction; 68 000 rows of 1003 columns (4163 spans)
+    take that path. Mask and skip list bit for bit against the oracle, with
+    16-byte aligned and misaligned buffers."""
+    binding = require_gpu()
+    lib = binding.load()
+    rows, cols, n_in = 68000, 1003, 8
+    rng = np.random.default_rng(68)
+    c_ref = rng.integers(0, n_in + 1, (rows, cols), dtype=np.int16)
+    m_ref = oracle.binarize_counts(c_ref, n_in, 0.5)
+    rp_ref, ci_ref = oracle.mask_rows_to_csr(m_ref[None])
+    dev = torch.device("cuda")
+    cells = rows * cols
+    for c_off, m_off in ((0, 0), (3, 5)):
+        cbuf = torch.zeros(cells + 8, dtype=torch.int16, device=dev)
+        cbuf[c_off:c_off + cells] = torch.from_numpy(c_ref.reshape(-1)).to(dev)
+        mbuf = torch.empty(cells + 16, dtype=torch.uint8, device=dev)
+        row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+        col_idx = torch.empty(cells, dtype=torch.int32, device=dev)
+        nnz = torch.zeros(1, dtype=torch.int64, device=dev)
+        ws = torch.empty(lib.calibatt_aggregate_rows_workspace_size(rows), dtype=torch.uint8, device=dev)
+        rc = lib.calibatt_aggregate_mask_rows(cbuf.data_ptr() + 2 * c_off, n_in, rows, cols, 0.5,
+                                              mbuf.data_ptr() + m_off, binding._ptr(row_ptr),
+                                              binding._ptr(col_idx), cells, binding._ptr(nnz), binding._ptr(ws),
+                                              ws.numel(), binding._stream(None))
+        assert rc == 0
+        torch.cuda.synchronize()
+        assert binding.get_status() == 0
+        np.testing.assert_array_equal(mbuf[m_off:m_off + cells].cpu().numpy().reshape(rows, cols), m_ref)
+        np.testing.assert_array_equal(row_ptr.cpu().numpy(), rp_ref)
+        total = int(nnz.item())
+        assert total == rp_ref[-1]
+        np.testing.assert_array_equal(col_idx[:total].cpu().numpy(), ci_ref)
+
+
 def test_aggregate_capacity_is_reported():
     binding = require_gpu()
     dev = torch.device("cuda")

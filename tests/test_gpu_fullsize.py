@@ -458,3 +458,42 @@ def test_calib720_sweep_40_heads_64_inputs(oracle):
         print(f"calib720 eps={eps}: block sparsity {1 - m_agg.mean():.4f}, {ties} tie-affected selections "
               f"at 1e-6 of {n_in * wl.heads * wl.nb}")
         del masks
+
+
+def test_aggregate_rows_near_the_cell_limit(oracle):
+    """The aggregation's flat indices and ranks are 32-bit (cells <= INT_MAX).
+    At 2^21 rows of 1023 columns (2 145 386 496 cells, within 2.1 M of the
+    limit; 4.3 GB of counts) every row's kept count is checked against the
+    oracle's binarisation, chunk by chunk on the host, and sampled rows (the
+    first, last and ones spread between) column by column; the mask is
+    compared in full."""
+    binding = require_gpu()
+    dev = torch.device("cuda")
+    rows, cols, n_in = 1 << 21, 1023, 100
+    assert rows * cols <= 2**31 - 1
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2024)
+    # counts in [0, 50]: about 2 % of the cells reach the threshold of 50
+    counts = torch.randint(0, 51, (rows, cols), device=dev, dtype=torch.int16, generator=gen).view(torch.uint16)
+    cap = 64 << 20
+    mask, row_ptr, col_idx, nnz = binding.aggregate_mask_rows(counts, n_in, 0.5, nnz_cap=cap, trim=False)
+    torch.cuda.synchronize()
+    assert binding.get_status() == 0
+    rp = row_ptr.cpu().numpy().astype(np.int64)
+    total = int(nnz.item())
+    assert rp[0] == 0 and rp[-1] == total and total < cap
+    chunk = 1 << 16
+    for r0 in range(0, rows, chunk):
+        c = counts[r0:r0 + chunk].view(torch.int16).cpu().numpy()
+        ref = oracle.binarize_counts(c, n_in, 0.5)
+        np.testing.assert_array_equal(mask[r0:r0 + chunk].cpu().numpy(), ref, err_msg=f"rows {r0}+")
+        np.testing.assert_array_equal(np.diff(rp[r0:r0 + chunk + 1]), ref.sum(1, dtype=np.int64), err_msg=f"rows {r0}+")
+    del c, ref
+    rng = np.random.default_rng(7)
+    sample = np.unique(np.concatenate([[0, 1, rows // 2, rows - 2, rows - 1], rng.integers(0, rows, 27)]))
+    ci = col_idx[:total]
+    for r in sample.tolist():
+        c = counts[r].view(torch.int16).cpu().numpy()
+        ref = oracle.binarize_counts(c[None], n_in, 0.5)[0]
+        np.testing.assert_array_equal(mask[r].cpu().numpy(), ref, err_msg=f"row {r}")
+        np.testing.assert_array_equal(ci[rp[r]:rp[r + 1]].cpu().numpy(), np.nonzero(ref)[0], err_msg=f"row {r}")
