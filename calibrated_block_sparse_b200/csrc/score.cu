@@ -13,11 +13,15 @@
 //             second pass would, and the row's tiles are reduced and selected
 //             as above. S is computed once instead of twice.
 //
-// CTA (320 threads, one per SM): two query-tile slots; warps 0-3 and 4-7 are
+// CTA (352 threads, one per SM): two query-tile slots; warps 0-3 and 4-7 are
 // the slots' row warpgroups (thread = query row = TMEM lane), warp 8 loads Q
-// and K tiles with TMA, warp 9 issues tcgen05.mma. Tensor memory holds two S
-// buffers per slot (4 x 128 columns), so the MMA of the next tile overlaps
-// the reduction of the current one.
+// and K tiles with TMA into one K ring per slot, warps 9 and 10 issue the
+// tcgen05.mma of slot 0 and slot 1. Tensor memory holds two S buffers per
+// slot (4 x 128 columns), so the MMA of the next tile overlaps the reduction
+// of the current one. One issuer per slot: a stage's barrier checks and
+// commits cost about as long as its eight MMAs, and with a single issuer the
+// tensor pipe waited through them; with two, one slot's bookkeeping overlaps
+// the other slot's MMAs.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -38,25 +42,27 @@
 namespace calibatt {
 namespace {
 
-constexpr int kScoreThreads = 320;
-constexpr int kScoreRing = 4;               // K tiles in flight
+constexpr int kScoreThreads = 352;
+constexpr int kSlotRing = 2;                // K tiles in flight per slot
 constexpr int kEnergyScratch = 16384;       // per slot: per-warp tile sums, then selection scratch
 // Pairs of a row whose 2^x goes to the FMA-pipe polynomial (bit i%8 of the
 // mask selects pair i) instead of MUFU; measured fastest with none.
 constexpr unsigned kScoreEmu = CALIBATT_SCORE_EMU;
 
+// Words the producer writes with each ring stage, read by the slot's issuer.
+constexpr uint32_t kStageFirst = 1;  // starts a unit: wait for its Q
+constexpr uint32_t kStageLast = 2;   // ends a unit: release its Q
+constexpr uint32_t kStageEnd = 4;    // no more tiles for this slot
+
 struct ScoreBarriers {
-  uint64_t ring_full[kScoreRing];
-  uint64_t ring_empty[kScoreRing];
+  uint64_t ring_full[2][kSlotRing];
+  uint64_t ring_empty[2][kSlotRing];
   uint64_t q_full[2];
   uint64_t q_empty[2];
   uint64_t s_full[2][2];
   uint64_t s_empty[2][2];
-  uint64_t mma_done;
-  uint32_t first[kScoreRing];  // ring stage starts a unit (wait for its Q)
-  uint32_t last[kScoreRing];   // ring stage ends a unit (release its Q)
-  uint32_t slot[kScoreRing];
-  uint32_t end;                // producer has no more tiles
+  uint64_t mma_done[2];
+  uint32_t flags[2][kSlotRing];
   uint32_t tmem_base;
   int abort;
 };
@@ -65,7 +71,7 @@ template <int MODE>
 struct ScoreLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTile;
-  static constexpr int kAuxOff = kRingOff + kScoreRing * kTile;
+  static constexpr int kAuxOff = kRingOff + 2 * kSlotRing * kTile;
   static constexpr int kAuxBytes = (MODE == kEnergy || MODE == kEnergy1) ? 2 * kEnergyScratch : 0;
   static constexpr int kBarOff = kAuxOff + kAuxBytes;
   static constexpr int kBytes = kBarOff + static_cast<int>(sizeof(ScoreBarriers));
@@ -95,10 +101,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int G = 2 * gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kScoreRing; ++i) {
-      mbar_init(&bar.ring_full[i], 1);
-      mbar_init(&bar.ring_empty[i], 1);
-    }
+    for (int s = 0; s < 2; ++s)
+      for (int i = 0; i < kSlotRing; ++i) {
+        mbar_init(&bar.ring_full[s][i], 1);
+        mbar_init(&bar.ring_empty[s][i], 1);
+      }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.q_full[s], 1);
       mbar_init(&bar.q_empty[s], 1);
@@ -107,7 +114,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         mbar_init(&bar.s_empty[s][b], 128);
       }
     }
-    mbar_init(&bar.mma_done, 1);
+    mbar_init(&bar.mma_done[0], 1);
+    mbar_init(&bar.mma_done[1], 1);
     bar.abort = 0;
     fence_barrier_init();
   }
@@ -126,7 +134,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       cur[s].round = 0;
       cursor_seek(p, 2 * blockIdx.x + s, G, cur[s]);
     }
-    uint32_t stage = 0, phase = 0, n_q[2] = {0, 0};
+    uint32_t stage[2] = {0, 0}, phase[2] = {0, 0}, n_q[2] = {0, 0};
     bool ok = true;
     while (ok && (cur[0].valid || cur[1].valid)) {
       for (int s = 0; s < 2 && ok; ++s) {
@@ -140,87 +148,89 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           tma_load_3d(dst + kHalf, &tm_q, &bar.q_full[s], 64, c.u.r * 128, c.u.hq);
           ++n_q[s];
         }
-        if (!(ok = mbar_wait<SW>(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns))) break;
-        bar.first[stage] = c.j == 0;
-        bar.last[stage] = c.j == c.u.nnz - 1;
-        bar.slot[stage] = s;
-        uint8_t* dst = smem + L::kRingOff + stage * kTile;
-        mbar_arrive_expect_tx(&bar.ring_full[stage], kTile);
-        tma_load_3d(dst, &tm_k, &bar.ring_full[stage], 0, c.j * 128, c.u.hkv);
-        tma_load_3d(dst + kHalf, &tm_k, &bar.ring_full[stage], 64, c.j * 128, c.u.hkv);
-        if (++stage == kScoreRing) {
-          stage = 0;
-          phase ^= 1;
+        const uint32_t st = stage[s];
+        if (!(ok = mbar_wait<SW>(&bar.ring_empty[s][st], phase[s] ^ 1, abort_flag, p.status, p.wait_limit_ns))) break;
+        bar.flags[s][st] = (c.j == 0 ? kStageFirst : 0u) | (c.j == c.u.nnz - 1 ? kStageLast : 0u);
+        uint8_t* dst = smem + L::kRingOff + (s * kSlotRing + st) * kTile;
+        mbar_arrive_expect_tx(&bar.ring_full[s][st], kTile);
+        tma_load_3d(dst, &tm_k, &bar.ring_full[s][st], 0, c.j * 128, c.u.hkv);
+        tma_load_3d(dst + kHalf, &tm_k, &bar.ring_full[s][st], 64, c.j * 128, c.u.hkv);
+        if (++stage[s] == kSlotRing) {
+          stage[s] = 0;
+          phase[s] ^= 1;
         }
         cursor_next(p, 2 * blockIdx.x + s, G, c);
       }
     }
-    bool marker = false;
-    if (ok && mbar_wait<SW>(&bar.ring_empty[stage], phase ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
-      bar.end = 1;
-      bar.slot[stage] = 2;  // end marker
-      mbar_arrive(&bar.ring_full[stage]);
-      marker = true;
-    }
-    // no copy may still be landing when the CTA leaves: wait for the latest
-    // phase of every ring stage and Q buffer. With the end marker sent, the
-    // latest phase of `stage` is the marker's own (its earlier copy was
-    // consumed before the producer could reuse the stage); without it (a
-    // wait failed), `stage` was not armed again and its latest phase is the
-    // previous lap's.
-    for (int i = 0; i < kScoreRing; ++i) {
-      int st = static_cast<int>(stage) - (marker ? 0 : 1) - i;
-      uint32_t ph = phase;
-      if (st < 0) {
-        st += kScoreRing;
-        ph ^= 1;
+    for (int s = 0; s < 2; ++s) {
+      const uint32_t st0 = stage[s], ph0 = phase[s];
+      bool marker = false;
+      if (ok && mbar_wait<SW>(&bar.ring_empty[s][st0], ph0 ^ 1, abort_flag, p.status, p.wait_limit_ns)) {
+        bar.flags[s][st0] = kStageEnd;
+        mbar_arrive(&bar.ring_full[s][st0]);
+        marker = true;
+      } else {
+        ok = false;
       }
-      volatile int never = 0;
-      mbar_wait(&bar.ring_full[st], ph, &never, p.status);
+      // no copy may still be landing when the CTA leaves: wait for the latest
+      // phase of every stage of this slot's ring. With the end marker sent,
+      // the latest phase of st0 is the marker's own (its earlier copy was
+      // consumed before the producer could reuse the stage); without it (a
+      // wait failed), st0 was not armed again and its latest phase is the
+      // previous lap's.
+      for (int i = 0; i < kSlotRing; ++i) {
+        int st = static_cast<int>(st0) - (marker ? 0 : 1) - i;
+        uint32_t ph = ph0;
+        if (st < 0) {
+          st += kSlotRing;
+          ph ^= 1;
+        }
+        volatile int never = 0;
+        mbar_wait(&bar.ring_full[s][st], ph, &never, p.status);
+      }
     }
     for (int s = 0; s < 2; ++s)
       if (n_q[s] > 0) {
         volatile int never = 0;
         mbar_wait(&bar.q_full[s], (n_q[s] - 1) & 1, &never, p.status);
       }
-  } else if (warp == 9 && lane == 0) {
-    // ---------------------------------------------------------- MMA issuer
-    uint32_t stage = 0, phase = 0, n_q[2] = {0, 0}, n_s[2] = {0, 0};
-    const uint64_t qdesc0 = desc_k_base(sbase + L::kQOff);
-    const uint64_t kdesc0 = desc_k_base(sbase + L::kRingOff);
+  } else if ((warp == 9 || warp == 10) && lane == 0) {
+    // ---------------------------------------------------------- MMA issuers, one per slot
+    const int s = warp - 9;
+    uint32_t stage = 0, phase = 0, n_q = 0, n_s = 0;
+    const uint64_t qd = desc_k_base(sbase + L::kQOff) + s * (kTile >> 4);
+    const uint64_t kdesc0 = desc_k_base(sbase + L::kRingOff) + s * kSlotRing * (kTile >> 4);
     while (true) {
-      if (!mbar_wait<SW>(&bar.ring_full[stage], phase, abort_flag, p.status, p.wait_limit_ns)) break;
-      // read every word of the stage now: once ring_empty is committed below,
-      // the producer may reuse the stage and rewrite them for its next tile
-      const uint32_t s = *reinterpret_cast<volatile uint32_t*>(&bar.slot[stage]);
-      if (s > 1) break;
-      const bool first = *reinterpret_cast<volatile uint32_t*>(&bar.first[stage]) != 0;
-      const bool last = *reinterpret_cast<volatile uint32_t*>(&bar.last[stage]) != 0;
-      if (first) {
-        if (!mbar_wait<SW>(&bar.q_full[s], n_q[s] & 1, abort_flag, p.status, p.wait_limit_ns)) break;
+      if (!mbar_wait<SW>(&bar.ring_full[s][stage], phase, abort_flag, p.status, p.wait_limit_ns)) break;
+      // read the stage's word now: once ring_empty is committed below, the
+      // producer may reuse the stage and rewrite it for its next tile
+      const uint32_t f = *reinterpret_cast<volatile uint32_t*>(&bar.flags[s][stage]);
+      if (f & kStageEnd) break;
+      if (f & kStageFirst) {
+        if (!mbar_wait<SW>(&bar.q_full[s], n_q & 1, abort_flag, p.status, p.wait_limit_ns)) break;
       }
-      const int buf = n_s[s] & 1;
-      if (!mbar_wait<SW>(&bar.s_empty[s][buf], ((n_s[s] >> 1) & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) break;
+      const int buf = n_s & 1;
+      if (!mbar_wait<SW>(&bar.s_empty[s][buf], ((n_s >> 1) & 1) ^ 1, abort_flag, p.status, p.wait_limit_ns)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + (2 * s + buf) * 128;
-      const uint64_t qd = qdesc0 + s * (kTile >> 4), kd = kdesc0 + stage * (kTile >> 4);
+      const uint64_t kd = kdesc0 + stage * (kTile >> 4);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) mma_ss(d_tmem, qd + desc_k_step(ks), kd + desc_k_step(ks), kIdescS, ks > 0);
-      mma_commit(&bar.ring_empty[stage]);
-      if (last) {
+      mma_commit(&bar.ring_empty[s][stage]);
+      if (f & kStageLast) {
         mma_commit(&bar.q_empty[s]);
-        ++n_q[s];
+        ++n_q;
       }
       mma_commit(&bar.s_full[s][buf]);
-      ++n_s[s];
-      if (++stage == kScoreRing) {
+      ++n_s;
+      if (++stage == kSlotRing) {
         stage = 0;
         phase ^= 1;
       }
     }
-    mma_commit(&bar.mma_done);
+    mma_commit(&bar.mma_done[s]);
     volatile int never = 0;
-    mbar_wait(&bar.mma_done, 0, &never, p.status);
+    mbar_wait(&bar.mma_done[s], 0, &never, p.status);
   } else if (warp < 8) {
     // ---------------------------------------------------------- row warpgroups
     // After a failed wait the warps keep walking their units with every wait
