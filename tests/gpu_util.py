@@ -51,7 +51,7 @@ def compare_masks(mask_gpu, mask_ref, affected):
 # floor for the probabilities below 2^-126 that ex2.approx.ftz flushes to zero.
 ENERGY_REL = 1e-5
 ENERGY_ABS = 1e-12
-NORTH_STAR_TIE = 1e-6  # the tie window when both sides select from the same energies
+SAME_ENERGY_TIE = 1e-6  # the tie window when both sides select from the same energies
 
 
 def energy_bound(E_ref):
@@ -74,7 +74,7 @@ def independent_tie_window(E_ref):
     closer than their two bounds: so a row whose cut lies within
     sum_c bound_c (plus the 1e-6 spec window) of eps, or whose energies
     at the cut are that close, may legitimately differ. Shape: rows."""
-    return energy_bound(E_ref).sum(-1) + NORTH_STAR_TIE
+    return energy_bound(E_ref).sum(-1) + SAME_ENERGY_TIE
 
 
 def cells_explained(agg_gpu, agg_ref, affected_rows):

@@ -17,7 +17,7 @@ import pytest
 import torch
 
 from calibrated_block_sparse_b200 import synth
-from gpu_util import (NORTH_STAR_TIE, attn_tolerance_ok, compare_masks, energy_ok, independent_tie_window,
+from gpu_util import (SAME_ENERGY_TIE, attn_tolerance_ok, compare_masks, energy_ok, independent_tie_window,
                       require_gpu, tie_affected)
 
 pytestmark = pytest.mark.gpu
@@ -55,7 +55,7 @@ def test_anchor_energy_and_selection_match_oracle(oracle, F, H, W, heads, rep, k
     assert ok, (worst, rel)
     np.testing.assert_allclose(E.sum(-1), 1.0, atol=1e-4)
     m_same, kept_same, cut = oracle.select(E, eps, with_cut=True)
-    aff = tie_affected(cut, eps, NORTH_STAR_TIE)
+    aff = tie_affected(cut, eps, SAME_ENERGY_TIE)
     assert compare_masks(mask.cpu().numpy(), m_same, aff)[2] == 0
     np.testing.assert_array_equal(kept.cpu().numpy()[~aff], kept_same[~aff])
     np.testing.assert_array_equal(tie.cpu().numpy().astype(bool), aff)

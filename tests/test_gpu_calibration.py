@@ -19,7 +19,7 @@ import pytest
 import torch
 
 from calibrated_block_sparse_b200 import synth
-from gpu_util import (NORTH_STAR_TIE, cells_explained, compare_masks, energy_ok, independent_tie_window,
+from gpu_util import (SAME_ENERGY_TIE, cells_explained, compare_masks, energy_ok, independent_tie_window,
                       require_gpu, tie_affected)
 
 pytestmark = pytest.mark.gpu
@@ -401,7 +401,7 @@ def test_radix_select_is_exact_on_hard_rows(oracle, nb):
     for eps in (0.0, 0.3 + 1 / 128, 0.84, 0.9, 0.99, 1.0, 1.5):
         mask, kept, _, tie = binding.select_mask(Ed, eps, tie=True)
         m_ref, kept_ref, cut = oracle.select(E.astype(np.float64), eps, with_cut=True)
-        aff = tie_affected(cut, eps, NORTH_STAR_TIE)
+        aff = tie_affected(cut, eps, SAME_ENERGY_TIE)
         n_diff, n_tie, bad = compare_masks(mask.cpu().numpy(), m_ref, aff)
         assert bad == 0, (eps, n_diff, n_tie)
         rows_ok = ~aff.reshape(-1)
@@ -437,10 +437,10 @@ def test_tie_flags_match_the_oracle_cut(oracle, nb):
             E[h, r] *= (eps + rng.uniform(-5e-7, 5e-7)) / cs[m]
     E = E.astype(np.float32)
     dev = torch.device("cuda")
-    mask, _, _, tie = binding.select_mask(torch.from_numpy(E).to(dev), eps, tie=True, tie_window=NORTH_STAR_TIE)
+    mask, _, _, tie = binding.select_mask(torch.from_numpy(E).to(dev), eps, tie=True, tie_window=SAME_ENERGY_TIE)
     _, _, cut = oracle.select(E.astype(np.float64), eps, with_cut=True)
-    aff = tie_affected(cut, eps, NORTH_STAR_TIE)
-    sure = _margin_ok(cut, eps, NORTH_STAR_TIE, 1e-12)
+    aff = tie_affected(cut, eps, SAME_ENERGY_TIE)
+    sure = _margin_ok(cut, eps, SAME_ENERGY_TIE, 1e-12)
     got = tie.cpu().numpy().astype(bool)
     assert aff.sum() > nb // 4  # the construction produced ties
     np.testing.assert_array_equal(got[sure], aff[sure])
@@ -448,6 +448,6 @@ def test_tie_flags_match_the_oracle_cut(oracle, nb):
     q, k, _ = synth.plain_qkv(2, 128 * 24 + 5, seed=nb)
     E2, _, _, _, t2 = binding.block_energy(q.to(dev), k.to(dev), eps=eps, tie=True)
     _, _, cut2 = oracle.select(E2.cpu().numpy().astype(np.float64), eps, with_cut=True)
-    sure2 = _margin_ok(cut2, eps, NORTH_STAR_TIE, 1e-12)
+    sure2 = _margin_ok(cut2, eps, SAME_ENERGY_TIE, 1e-12)
     np.testing.assert_array_equal(t2.cpu().numpy().astype(bool)[sure2],
-                                  tie_affected(cut2, eps, NORTH_STAR_TIE)[sure2])
+                                  tie_affected(cut2, eps, SAME_ENERGY_TIE)[sure2])

@@ -33,7 +33,7 @@ import pytest
 import torch
 
 from calibrated_block_sparse_b200 import synth
-from gpu_util import (NORTH_STAR_TIE, attn_tolerance_ok, compare_masks, energy_ok, independent_tie_window,
+from gpu_util import (SAME_ENERGY_TIE, attn_tolerance_ok, compare_masks, energy_ok, independent_tie_window,
                       require_gpu, tie_affected)
 
 pytestmark = pytest.mark.gpu
@@ -320,8 +320,8 @@ def test_single_pass_energy_full_size(oracle, name):
         assert _energy_ok(E[h][brs], E_ref[i]), (name, h)
         np.testing.assert_allclose(E[h][brs].sum(-1), 1.0, atol=1e-4)
         m_same, _, cut = oracle.select(E[h][brs], eps, with_cut=True)
-        assert compare_masks(mask[h][brs], m_same, tie_affected(cut, eps, NORTH_STAR_TIE))[2] == 0
-        np.testing.assert_array_equal(tie[h][brs], tie_affected(cut, eps, NORTH_STAR_TIE))
+        assert compare_masks(mask[h][brs], m_same, tie_affected(cut, eps, SAME_ENERGY_TIE))[2] == 0
+        np.testing.assert_array_equal(tie[h][brs], tie_affected(cut, eps, SAME_ENERGY_TIE))
         m_ref, _, cut_ref = oracle.select(E_ref[i], eps, with_cut=True)
         assert compare_masks(mask[h][brs], m_ref, tie_affected(cut_ref, eps, independent_tie_window(E_ref[i])))[2] == 0
     print(f"{name}: {int(tie.sum())} of {tie.size} block-rows tie-affected at 1e-6")
@@ -434,7 +434,7 @@ def test_calib720_sweep_40_heads_64_inputs(oracle):
                 m_same, _, cut = oracle.select(Eg, eps, with_cut=True)
                 m_g, _, _ = binding.select_mask(E, eps, kept=False)
                 mg = m_g.cpu().numpy()[hs][:, brs].reshape(-1, wl.nb)
-                assert compare_masks(mg, m_same, tie_affected(cut, eps, NORTH_STAR_TIE))[2] == 0
+                assert compare_masks(mg, m_same, tie_affected(cut, eps, SAME_ENERGY_TIE))[2] == 0
                 m_ref, _, cut_ref = oracle.select(E_ref, eps, with_cut=True)
                 assert compare_masks(mg, m_ref, tie_affected(cut_ref, eps, independent_tie_window(E_ref)))[2] == 0
     assert binding.get_status() == 0
